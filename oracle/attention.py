@@ -1,0 +1,270 @@
+"""Plain float64 CPU definition of exact (ring) attention -- test infrastructure.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+legs may use this module.  It is deliberately slow and literal:
+
+* ``attention_ref`` is the textbook definition, one full score row per query
+  (the attention definition on the pages [BT] "core challenge", [LC] "the
+  mathematical essence of attention", [RA] §2.3), with the readings below.
+* ``ring_ref`` / ``block_step_ref`` / ``finalize_ref`` follow the ring
+  algorithm step by step: cut the sequence into P chunks ([RA] §2.1), let
+  query chunk i visit KV chunk (i+s) mod P at step s ([RA] §2.2 figure), fold
+  each visit into running (acc, m, l) statistics ([RA] §3.1 inner loop,
+  "softmax in SRAM"), then normalise once over all keys ([LC] fusion layer:
+  global softmax normalisation of the local outputs).
+* ``lse_merge_ref`` combines independently normalised partials by their
+  log-sum-exp weights (the same global normalisation, [LC] fusion layer).
+
+Readings where the pages are silent or wrong (each listed in the design notes):
+  - [RA] §2.3 writes the sum of independently normalised per-chunk softmaxes;
+    taken literally that is not attention.  The sentence after it says the
+    accumulated result *is* full attention, and [LC] normalises globally, so
+    the merge here is the global softmax over all keys.
+  - causal masking is per token (causal_block_size=1 in [CI]): key position
+    k_pos is visible to query position q_pos iff k_pos <= q_pos.
+  - cache_idx = -1 means "None": query t sits at global position t.
+    cache_idx >= 0: query t sits at cache_idx + t (the exact offset; [CI]
+    floors it to a query-chunk multiple, identical whenever cache_idx is a
+    multiple of the query chunk).
+  - GQA (not on the pages): query head h reads KV head h // (Hq // Hkv).
+  - a masked logit is -inf; a row with no visible key has out = 0, lse = -inf;
+    an all-masked visit leaves the running state unchanged.
+  - lse is the natural log of sum_j exp(scale * q.k_j) over visible keys.
+
+Array layouts (token-major): q/out [B, N_q, Hq, d]; k/v [B, N_kv, Hkv, d];
+lse [B, Hq, N_q]; running state acc [B, Hq, Lq, d], m and l [B, Hq, Lq];
+split partials o_parts [S, B, N_q, Hq, d], lse_parts [S, B, Hq, N_q].
+"""
+from __future__ import annotations
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+# Rows of queries per dense score block in attention_ref.  Rows are
+# independent, so this only bounds memory; each row still sees its whole
+# score row at once.
+_ROW_BLOCK = 256
+
+
+def _f64(x) -> np.ndarray:
+    """Upcast a torch tensor (any float dtype, any device) or array to float64."""
+    if hasattr(x, "detach"):
+        import torch
+        return x.detach().cpu().to(dtype=torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _kv_head(h_q: int, Hq: int, Hkv: int) -> int:
+    """Query head h_q reads KV head h_q // G with G = Hq / Hkv (contiguous groups)."""
+    return h_q // (Hq // Hkv)
+
+
+def _query_positions(N_q: int, cache_idx: int) -> np.ndarray:
+    """Global token position of each query row ([CI] "how cache_idx works")."""
+    base = 0 if cache_idx < 0 else int(cache_idx)
+    return base + np.arange(N_q, dtype=np.int64)
+
+
+def _visible(q_pos: np.ndarray, k_pos: np.ndarray, causal: bool) -> np.ndarray:
+    """[len(q_pos), len(k_pos)] boolean: may query q_pos attend to key k_pos?"""
+    if not causal:
+        return np.ones((q_pos.shape[0], k_pos.shape[0]), dtype=bool)
+    return k_pos[None, :] <= q_pos[:, None]
+
+
+def _softmax_rows(s: np.ndarray):
+    """Stable softmax statistics of score rows that may hold -inf entries.
+
+    Returns (w, m, l): w = exp(s - m) with m the row max (0 used as the
+    subtraction base for rows that are entirely -inf), l = row sum of w.
+    """
+    m = s.max(axis=1)
+    base = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(s - base[:, None])
+    l = w.sum(axis=1)
+    return w, m, l
+
+
+def attention_ref(q, k, v, *, causal: bool, scale: float, cache_idx: int = -1,
+                  rows=None, heads=None):
+    """Exact attention by definition, in float64.
+
+    out[b, t, h, :] = sum_j softmax_j(scale * q[b,t,h,:] . k[b,j,hk,:]) v[b,j,hk,:]
+    over the keys j visible to row t, and lse[b, h, t] = log sum_j exp(...).
+
+    ``rows`` (query indices) and ``heads`` (query heads) restrict the
+    computation to a sample; the returned arrays then have len(rows) rows
+    and len(heads) heads in the order given.
+    Returns (out [B, R, Hh, d], lse [B, Hh, R]) as float64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N_q, Hq, d = q.shape
+    N_kv, Hkv = k.shape[1], k.shape[2]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    rows = np.arange(N_q) if rows is None else np.asarray(rows, dtype=np.int64)
+    heads = list(range(Hq)) if heads is None else list(heads)
+    pos_all = _query_positions(N_q, cache_idx)
+    out = np.zeros((B, rows.shape[0], len(heads), d), dtype=np.float64)
+    lse = np.full((B, len(heads), rows.shape[0]), NEG_INF, dtype=np.float64)
+    k_pos_all = np.arange(N_kv, dtype=np.int64)
+    for b in range(B):
+        for hi, h in enumerate(heads):
+            hk = _kv_head(h, Hq, Hkv)
+            for r0 in range(0, rows.shape[0], _ROW_BLOCK):
+                r = rows[r0:r0 + _ROW_BLOCK]
+                qp = pos_all[r]
+                # Keys past the last query position carry zero weight under
+                # causal masking; leave them out of the product.
+                n_keys = N_kv if not causal else int(min(N_kv, qp.max() + 1))
+                if n_keys <= 0:
+                    continue
+                s = scale * (q[b, r, h, :] @ k[b, :n_keys, hk, :].T)
+                s = np.where(_visible(qp, k_pos_all[:n_keys], causal), s, NEG_INF)
+                w, m, l = _softmax_rows(s)
+                has = l > 0
+                o = np.zeros((r.shape[0], d))
+                o[has] = (w[has] @ v[b, :n_keys, hk, :]) / l[has, None]
+                out[b, r0:r0 + r.shape[0], hi, :] = o
+                lse[b, hi, r0:r0 + r.shape[0]] = np.where(
+                    has, m + np.log(np.where(has, l, 1.0)), NEG_INF)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# The ring algorithm, step by step.
+# ---------------------------------------------------------------------------
+
+def ring_visit_chunk(i: int, s: int, P: int, direction: int = 1) -> int:
+    """KV chunk held by query chunk i at ring step s.
+
+    direction=+1: (i + s) mod P, the schedule of the [RA] §2.2 figure
+    (GPU0 receives K1, K2, K3 at steps 1, 2, 3).  direction=-1: (i - s) mod P,
+    what a ring that sends to (i+1) mod n delivers ([CI] ppermute, [BT]).
+    """
+    return (i + direction * s) % P
+
+
+def query_home_chunk(q_pos0: int, chunk: int) -> int:
+    """Ring rank whose chunk holds global position q_pos0 (the block's first query)."""
+    return int(q_pos0) // int(chunk)
+
+
+def init_state(B: int, Hq: int, Lq: int, d: int):
+    """Empty running statistics: acc = 0, m = -inf, l = 0."""
+    return (np.zeros((B, Hq, Lq, d)), np.full((B, Hq, Lq), NEG_INF), np.zeros((B, Hq, Lq)))
+
+
+def block_step_ref(q_chunk, k_chunk, v_chunk, q_off: int, k_off: int, acc, m, l, *,
+                   causal: bool, scale: float):
+    """Fold one ring visit (a query chunk against one KV chunk) into (acc, m, l).
+
+    q_chunk [B, Lq, Hq, d] at global positions q_off + t; k/v_chunk
+    [B, Lk, Hkv, d] at k_off + j.  m is in natural-log units of
+    scale * q.k.  Per row: m' = max(m, max_j s_j), alpha = exp(m - m'),
+    l' = alpha l + sum_j exp(s_j - m'), acc' = alpha acc + sum_j exp(s_j - m') v_j.
+    Returns new (acc, m, l); the inputs are not modified.
+    """
+    q, kc, vc = _f64(q_chunk), _f64(k_chunk), _f64(v_chunk)
+    acc, m, l = (np.array(_f64(x), copy=True) for x in (acc, m, l))
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = kc.shape[1], kc.shape[2]
+    vis = _visible(q_off + np.arange(Lq, dtype=np.int64),
+                   k_off + np.arange(Lk, dtype=np.int64), causal)
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            s = scale * (q[b, :, h, :] @ kc[b, :, hk, :].T)
+            s = np.where(vis, s, NEG_INF)
+            m_new = np.maximum(m[b, h], s.max(axis=1) if Lk > 0 else NEG_INF)
+            base = np.where(np.isfinite(m_new), m_new, 0.0)
+            alpha = np.exp(m[b, h] - base)
+            p = np.exp(s - base[:, None])
+            l[b, h] = alpha * l[b, h] + p.sum(axis=1)
+            acc[b, h] = alpha[:, None] * acc[b, h] + p @ vc[b, :, hk, :]
+            m[b, h] = m_new
+    return acc, m, l
+
+
+def finalize_ref(acc, m, l):
+    """out = acc / l, lse = m + log l; rows with l == 0 give out 0 and lse -inf.
+
+    Returns (out [B, Lq, Hq, d], lse [B, Hq, Lq]).
+    """
+    acc, m, l = _f64(acc), _f64(m), _f64(l)
+    has = l > 0
+    safe = np.where(has, l, 1.0)
+    out = np.where(has[..., None], acc / safe[..., None], 0.0)
+    lse = np.where(has, m + np.log(safe), NEG_INF)
+    return np.transpose(out, (0, 2, 1, 3)), lse
+
+
+def ring_ref(q, k, v, *, causal: bool, scale: float, P: int, chunk: int, cache_idx: int = -1,
+             order="forward"):
+    """Ring attention emulated on the CPU: every query block visits all P KV chunks.
+
+    Prefill (cache_idx = -1): query chunk i holds rows [i*chunk, (i+1)*chunk)
+    and starts from KV chunk i.  Incremental (cache_idx >= 0): all N_q new
+    queries form one block homed at the chunk holding position cache_idx.
+    ``order`` picks the visit sequence: "forward" (i+s) mod P, "backward"
+    (i-s) mod P, or an explicit permutation of range(P) (same for every block).
+    Returns (out [B, N_q, Hq, d], lse [B, Hq, N_q]) in float64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N_q, Hq, d = q.shape
+    N_kv = k.shape[1]
+    if P * chunk != N_kv:
+        raise ValueError("N_kv must equal P * chunk")
+    if cache_idx < 0:
+        if N_q != N_kv:
+            raise ValueError("prefill needs N_q == N_kv")
+        blocks = [(i, i * chunk, slice(i * chunk, (i + 1) * chunk)) for i in range(P)]
+    else:
+        blocks = [(query_home_chunk(cache_idx, chunk), int(cache_idx), slice(0, N_q))]
+
+    def visits(i):
+        if isinstance(order, str):
+            direction = {"forward": 1, "backward": -1}[order]
+            return [ring_visit_chunk(i, s, P, direction) for s in range(P)]
+        seq = [int(x) for x in order]
+        if sorted(seq) != list(range(P)):
+            raise ValueError("order must be a permutation of range(P)")
+        return seq
+
+    out = np.zeros((B, N_q, Hq, d))
+    lse = np.zeros((B, Hq, N_q))
+    for i, q_off, rs in blocks:
+        qb = q[:, rs]
+        acc, m, l = init_state(B, Hq, qb.shape[1], d)
+        for j in visits(i):
+            ks = slice(j * chunk, (j + 1) * chunk)
+            acc, m, l = block_step_ref(qb, k[:, ks], v[:, ks], q_off, j * chunk, acc, m, l,
+                                       causal=causal, scale=scale)
+        ob, lb = finalize_ref(acc, m, l)
+        out[:, rs] = ob
+        lse[:, :, rs] = lb
+    return out, lse
+
+
+def lse_merge_ref(o_parts, lse_parts):
+    """Merge S normalised partial results by their log-sum-exp weights.
+
+    o_parts [S, B, N_q, Hq, d], lse_parts [S, B, Hq, N_q].  Per row:
+    M = max_s lse_s, w_s = exp(lse_s - M), lse = M + log sum_s w_s,
+    out = sum_s w_s O_s / sum_s w_s.  A partial with lse = -inf has weight 0;
+    a row whose partials are all -inf gives out 0 and lse -inf.
+    Returns (out [B, N_q, Hq, d], lse [B, Hq, N_q]).
+    """
+    o, L = _f64(o_parts), _f64(lse_parts)
+    M = L.max(axis=0)
+    base = np.where(np.isfinite(M), M, 0.0)
+    w = np.exp(L - base[None])                    # [S, B, Hq, N_q]
+    W = w.sum(axis=0)
+    has = W > 0
+    safe = np.where(has, W, 1.0)
+    w_t = np.transpose(w, (0, 1, 3, 2))[..., None]  # [S, B, N_q, Hq, 1]
+    out = (w_t * o).sum(axis=0) / np.transpose(safe, (0, 2, 1))[..., None]
+    out = np.where(np.transpose(has, (0, 2, 1))[..., None], out, 0.0)
+    lse = np.where(has, base + np.log(safe), NEG_INF)
+    return out, lse

@@ -1,0 +1,320 @@
+"""Pins that tie the CPU oracle to things other than itself.
+
+Each ``pin_*`` takes the oracle module ``O`` (the real ``oracle.attention`` or
+a deliberately broken copy) and raises AssertionError on a mismatch.  The
+pins use: torch's float64 scaled_dot_product_attention and logsumexp (library
+routines independent of the oracle's NumPy code), brute force in pure-Python
+scalar loops, closed forms, invariants of the method, and the ring schedule
+printed in the pages' figure (``tests/golden/ring_schedule.json``).
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TOL = 1e-11
+
+
+def _rand(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float64) * scale)
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    fin = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), fin), f"{what}: finiteness differs"
+    assert np.array_equal(a[~fin], b[~fin]), f"{what}: infinities differ"
+    err = np.max(np.abs(a[fin] - b[fin])) if fin.any() else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+
+
+def _sdpa_case(q, k, v, causal, scale, cache_idx):
+    """torch SDPA in float64 with an explicit boolean mask; GQA by repeating KV heads."""
+    B, N_q, Hq, d = q.shape
+    N_kv, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    kr = k.repeat_interleave(G, dim=2)
+    vr = v.repeat_interleave(G, dim=2)
+    qpos = torch.arange(N_q) + (0 if cache_idx < 0 else cache_idx)
+    kpos = torch.arange(N_kv)
+    mask = (kpos[None, :] <= qpos[:, None]) if causal else torch.ones(N_q, N_kv, dtype=torch.bool)
+    out = F.scaled_dot_product_attention(q.transpose(1, 2), kr.transpose(1, 2), vr.transpose(1, 2),
+                                         attn_mask=mask, scale=scale).transpose(1, 2)
+    s = torch.einsum("bqhd,bkhd->bhqk", q, kr) * scale
+    s = s.masked_fill(~mask, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return out.numpy(), lse.numpy()
+
+
+SDPA_CASES = [
+    # (B, N_q, N_kv, Hq, Hkv, d, causal, scale, cache_idx)
+    (2, 37, 37, 3, 3, 16, False, 0.25, -1),
+    (1, 50, 50, 2, 2, 8, True, 1 / math.sqrt(8), -1),
+    (2, 7, 27, 4, 4, 16, True, 0.3, 20),
+    (1, 33, 33, 6, 2, 8, True, 0.35, -1),
+    (1, 5, 40, 4, 1, 8, False, 0.2, 35),
+]
+
+
+def pin_sdpa(O):
+    for i, (B, N_q, N_kv, Hq, Hkv, d, causal, scale, ci) in enumerate(SDPA_CASES):
+        q = _rand((B, N_q, Hq, d), 10 + i)
+        k = _rand((B, N_kv, Hkv, d), 20 + i)
+        v = _rand((B, N_kv, Hkv, d), 30 + i)
+        ref_o, ref_l = _sdpa_case(q, k, v, causal, scale, ci)
+        o, l = O.attention_ref(q, k, v, causal=causal, scale=scale, cache_idx=ci)
+        _close(o, ref_o, 1e-10, f"sdpa out case {i}")
+        _close(l, ref_l, 1e-10, f"sdpa lse case {i}")
+
+
+def _brute(q, k, v, causal, scale, cache_idx):
+    """Scalar loops straight from the definition (tiny sizes only)."""
+    q, k, v = q.tolist(), k.tolist(), v.tolist()
+    B, N_q, Hq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    N_kv, Hkv = len(k[0]), len(k[0][0])
+    G = Hq // Hkv
+    out = [[[[0.0] * d for _ in range(Hq)] for _ in range(N_q)] for _ in range(B)]
+    lse = [[[0.0] * N_q for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            for t in range(N_q):
+                pos = t if cache_idx < 0 else cache_idx + t
+                keys = [j for j in range(N_kv) if (not causal or j <= pos)]
+                sc = [scale * sum(q[b][t][h][e] * k[b][j][hk][e] for e in range(d)) for j in keys]
+                mx = max(sc)
+                ws = [math.exp(x - mx) for x in sc]
+                tot = sum(ws)
+                for e in range(d):
+                    out[b][t][h][e] = sum(w * v[b][j][hk][e] for w, j in zip(ws, keys)) / tot
+                lse[b][h][t] = mx + math.log(tot)
+    return np.array(out), np.array(lse)
+
+
+def pin_bruteforce(O):
+    cases = [(1, 6, 6, 2, 1, 3, True, 0.7, -1), (2, 5, 5, 2, 2, 4, False, 0.5, -1),
+             (1, 3, 9, 3, 1, 2, True, 1.1, 6)]
+    for i, (B, N_q, N_kv, Hq, Hkv, d, causal, scale, ci) in enumerate(cases):
+        q = _rand((B, N_q, Hq, d), 40 + i)
+        k = _rand((B, N_kv, Hkv, d), 50 + i)
+        v = _rand((B, N_kv, Hkv, d), 60 + i)
+        bo, bl = _brute(q, k, v, causal, scale, ci)
+        o, l = O.attention_ref(q, k, v, causal=causal, scale=scale, cache_idx=ci)
+        _close(o, bo, 1e-12, f"brute out {i}")
+        _close(l, bl, 1e-12, f"brute lse {i}")
+
+
+def pin_closed_forms(O):
+    N, d, scale = 24, 8, 0.4
+    v = _rand((1, N, 1, d), 70)
+    # Identical keys: every visible key has the same score s, so the output is
+    # the plain mean of the visible values and lse = s + ln(#visible).
+    q = _rand((1, N, 1, d), 71)
+    k1 = _rand((1, 1, 1, d), 72)
+    k = k1.expand(1, N, 1, d).contiguous()
+    o, l = O.attention_ref(q, k, v, causal=True, scale=scale)
+    vv = v[0, :, 0].numpy()
+    cnt = np.arange(1, N + 1)
+    prefix_mean = np.cumsum(vv, axis=0) / cnt[:, None]
+    s = scale * (q[0, :, 0] @ k1[0, 0, 0]).numpy()
+    _close(o[0, :, 0], prefix_mean, 1e-12, "identical keys out")
+    _close(l[0, 0], s + np.log(cnt), 1e-12, "identical keys lse")
+    # Non-causal identical keys: mean over all values.
+    o, l = O.attention_ref(q, k, v, causal=False, scale=scale)
+    _close(o[0, :, 0], np.broadcast_to(vv.mean(axis=0), (N, d)), 1e-12, "identical keys mean")
+    _close(l[0, 0], s + np.log(N), 1e-12, "identical keys lse all")
+    # A single key returns its value; lse is its score.
+    o, l = O.attention_ref(q[:, :5], k1, v[:, :1], causal=False, scale=scale)
+    _close(o[0, :, 0], np.broadcast_to(vv[0], (5, d)), 1e-14, "single key out")
+    _close(l[0, 0], scale * (q[0, :5, 0] @ k1[0, 0, 0]).numpy(), 1e-12, "single key lse")
+    # Causal row 0 sees only key 0.
+    kk = _rand((1, N, 1, d), 73)
+    o, l = O.attention_ref(q, kk, v, causal=True, scale=scale)
+    _close(o[0, 0, 0], vv[0], 1e-14, "causal row 0")
+    _close(l[0, 0, 0], scale * float(q[0, 0, 0] @ kk[0, 0, 0]), 1e-12, "causal row 0 lse")
+    # scale = 0: uniform weights -> prefix mean, lse = ln(t + 1).
+    o, l = O.attention_ref(q, kk, v, causal=True, scale=0.0)
+    _close(o[0, :, 0], prefix_mean, 1e-12, "scale 0 out")
+    _close(l[0, 0], np.log(cnt), 1e-12, "scale 0 lse")
+    # A dominant key: orthonormal keys and q = 60 e_j pick v_j.
+    kd = torch.eye(d, dtype=torch.float64).reshape(1, d, 1, d)
+    vd = _rand((1, d, 1, d), 74)
+    j = 5
+    qd = torch.zeros(1, 1, 1, d, dtype=torch.float64)
+    qd[0, 0, 0, j] = 60.0
+    o, l = O.attention_ref(qd, kd, vd, causal=False, scale=1.0)
+    _close(o[0, 0, 0], vd[0, j, 0].numpy(), 1e-12, "dominant key")
+    _close(l[0, 0, 0], 60.0 + np.log1p((d - 1) * np.exp(-60.0)), 1e-12, "dominant key lse")
+
+
+def pin_ring_equals_full(O):
+    rng = np.random.default_rng(3)
+    N, d = 64, 8
+    for causal in (True, False):
+        for Hq, Hkv in ((2, 2), (4, 2)):
+            q = _rand((2, N, Hq, d), 80)
+            k = _rand((2, N, Hkv, d), 81)
+            v = _rand((2, N, Hkv, d), 82)
+            fo, fl = O.attention_ref(q, k, v, causal=causal, scale=0.3)
+            for P in (1, 2, 4, 8, 16):
+                orders = ["forward", "backward", list(rng.permutation(P))]
+                for order in orders:
+                    ro, rl = O.ring_ref(q, k, v, causal=causal, scale=0.3, P=P, chunk=N // P,
+                                        order=order)
+                    _close(ro, fo, 1e-12, f"ring P={P} {order} causal={causal}")
+                    _close(rl, fl, 1e-12, f"ring lse P={P} {order}")
+    # Incremental queries through the ring.
+    N_kv, N_q, ci = 64, 10, 50
+    q = _rand((1, N_q, 2, d), 83)
+    k = _rand((1, N_kv, 1, d), 84)
+    v = _rand((1, N_kv, 1, d), 85)
+    fo, fl = O.attention_ref(q, k, v, causal=True, scale=0.3, cache_idx=ci)
+    for P in (1, 4, 8):
+        for order in ("forward", "backward", list(rng.permutation(P))):
+            ro, rl = O.ring_ref(q, k, v, causal=True, scale=0.3, P=P, chunk=N_kv // P,
+                                cache_idx=ci, order=order)
+            _close(ro, fo, 1e-12, f"ring cache_idx P={P} {order}")
+            _close(rl, fl, 1e-12, f"ring cache_idx lse P={P} {order}")
+
+
+def pin_invariants(O):
+    N, d = 40, 8
+    q = _rand((3, N, 4, d), 90)
+    k = _rand((3, N, 2, d), 91)
+    v = _rand((3, N, 2, d), 92)
+    fo, fl = O.attention_ref(q, k, v, causal=True, scale=0.3)
+    # cache_idx rows equal the matching rows of full causal prefill.
+    for c in (0, 1, 17, 39):
+        co, cl = O.attention_ref(q[:, c:], k, v, causal=True, scale=0.3, cache_idx=c)
+        _close(co, fo[:, c:], 1e-12, f"cache_idx {c} out")
+        _close(cl, fl[:, :, c:], 1e-12, f"cache_idx {c} lse")
+    # GQA with KV heads replicated into MHA gives the same result.
+    mo, ml = O.attention_ref(q, k.repeat_interleave(2, dim=2), v.repeat_interleave(2, dim=2),
+                             causal=True, scale=0.3)
+    _close(mo, fo, 1e-12, "gqa vs mha")
+    _close(ml, fl, 1e-12, "gqa vs mha lse")
+    # Batches are independent.
+    bo, bl = O.attention_ref(q[1:2], k[1:2], v[1:2], causal=True, scale=0.3)
+    _close(bo, fo[1:2], 1e-12, "batch independence")
+    # Non-causal: permuting (K, V) jointly leaves the result unchanged.
+    no, nl = O.attention_ref(q, k, v, causal=False, scale=0.3)
+    perm = torch.randperm(N, generator=torch.Generator().manual_seed(5))
+    po, pl = O.attention_ref(q, k[:, perm], v[:, perm], causal=False, scale=0.3)
+    _close(po, no, 1e-12, "kv permutation")
+    _close(pl, nl, 1e-12, "kv permutation lse")
+    # Causal differs from non-causal except on the last row.
+    assert np.max(np.abs(no[:, :-1] - fo[:, :-1])) > 1e-3, "causal mask has no effect"
+    _close(no[:, -1], fo[:, -1], 1e-12, "last row sees every key")
+
+
+def pin_block_step(O):
+    # One visit then finalize equals attention over that chunk; an all-masked
+    # visit leaves the state unchanged.
+    B, Lq, Lk, Hq, Hkv, d = 2, 6, 9, 4, 2, 8
+    q = _rand((B, Lq, Hq, d), 100)
+    k = _rand((B, Lk, Hkv, d), 101)
+    v = _rand((B, Lk, Hkv, d), 102)
+    acc, m, l = O.init_state(B, Hq, Lq, d)
+    acc, m, l = O.block_step_ref(q, k, v, 0, 0, acc, m, l, causal=False, scale=0.5)
+    o, ls = O.finalize_ref(acc, m, l)
+    ro, rl = O.attention_ref(q, k, v, causal=False, scale=0.5)
+    _close(o, ro, 1e-12, "single visit")
+    _close(ls, rl, 1e-12, "single visit lse")
+    a2, m2, l2 = O.block_step_ref(q, k, v, 0, 100, acc, m, l, causal=True, scale=0.5)
+    _close(a2, acc, 0.0, "masked visit acc")
+    _close(m2, m, 0.0, "masked visit m")
+    _close(l2, l, 0.0, "masked visit l")
+    # From the empty state an all-masked visit stays empty: out 0, lse -inf.
+    e = O.init_state(B, Hq, Lq, d)
+    a3, m3, l3 = O.block_step_ref(q, k, v, 0, 100, *e, causal=True, scale=0.5)
+    o3, ls3 = O.finalize_ref(a3, m3, l3)
+    assert np.all(o3 == 0) and np.all(np.isneginf(ls3)), "empty row"
+    # Causal diagonal visit equals causal attention of the chunk with itself.
+    k2 = _rand((B, Lq, Hkv, d), 103)
+    v2 = _rand((B, Lq, Hkv, d), 104)
+    acc, m, l = O.block_step_ref(q, k2, v2, 7, 7, *O.init_state(B, Hq, Lq, d), causal=True,
+                                 scale=0.5)
+    o, ls = O.finalize_ref(acc, m, l)
+    ro, rl = O.attention_ref(q, k2, v2, causal=True, scale=0.5)
+    _close(o, ro, 1e-12, "diagonal visit")
+    _close(ls, rl, 1e-12, "diagonal visit lse")
+
+
+def pin_lse_merge(O):
+    # Split the keys of a non-causal problem into disjoint sets; attention over
+    # each set gives normalised partials whose merge is attention over all keys.
+    B, N_q, N_kv, Hq, d = 2, 7, 30, 3, 8
+    q = _rand((B, N_q, Hq, d), 110)
+    k = _rand((B, N_kv, Hq, d), 111)
+    v = _rand((B, N_kv, Hq, d), 112)
+    full_o, full_l = O.attention_ref(q, k, v, causal=False, scale=0.4)
+    cuts = [0, 4, 13, 22, 30]
+    parts = [O.attention_ref(q, k[:, a:b], v[:, a:b], causal=False, scale=0.4)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    po = np.stack([p[0] for p in parts])
+    pl = np.stack([p[1] for p in parts])
+    mo, ml = O.lse_merge_ref(po, pl)
+    _close(mo, full_o, 1e-12, "merge = full")
+    _close(ml, full_l, 1e-12, "merge lse = full")
+    # Commutative: any order of partials.
+    for perm in itertools.permutations(range(4)):
+        co, cl = O.lse_merge_ref(po[list(perm)], pl[list(perm)])
+        _close(co, mo, 1e-12, "merge commutative")
+        _close(cl, ml, 1e-12, "merge commutative lse")
+    # Associative: merging merged groups gives the same answer.
+    ao, al = O.lse_merge_ref(po[:2], pl[:2])
+    bo, bl = O.lse_merge_ref(po[2:], pl[2:])
+    to, tl = O.lse_merge_ref(np.stack([ao, bo]), np.stack([al, bl]))
+    _close(to, mo, 1e-12, "merge associative")
+    _close(tl, ml, 1e-12, "merge associative lse")
+    # Identity: a partial with lse = -inf (no keys) changes nothing.
+    io, il = O.lse_merge_ref(np.stack([po[0], np.full_like(po[0], 123.0)]),
+                             np.stack([pl[0], np.full_like(pl[0], -np.inf)]))
+    _close(io, po[0], 1e-14, "merge identity")
+    _close(il, pl[0], 1e-14, "merge identity lse")
+    # All partials empty: out 0, lse -inf.
+    eo, el = O.lse_merge_ref(np.ones((2, 1, 2, 1, 4)), np.full((2, 1, 1, 2), -np.inf))
+    assert np.all(eo == 0) and np.all(np.isneginf(el)), "merge of empties"
+
+
+def pin_schedule(O):
+    g = json.load(open(os.path.join(GOLDEN, "ring_schedule.json")))
+    fig = g["figure_4gpu"]
+    for e in fig["entries"]:
+        got = O.ring_visit_chunk(e["gpu"], e["step"], fig["P"], 1)
+        assert got == e["chunk"], f"figure: step {e['step']} gpu {e['gpu']} -> {got}"
+    for e in fig["inconsistent_entries"]:
+        # Garbled entry: neither direction reproduces it at the printed step.
+        assert O.ring_visit_chunk(e["gpu"], e["step"], fig["P"], 1) != e["chunk"]
+        assert O.ring_visit_chunk(e["gpu"], e["step"], fig["P"], -1) != e["chunk"]
+    # ppermute ring: simulate the sends and compare with direction -1.
+    pr = g["ppermute_ring"]
+    n = pr["n"]
+    holding = list(range(n))
+    for s in range(1, n):
+        new = [None] * n
+        for src, dst in pr["perm"]:
+            new[dst] = holding[src]
+        holding = new
+        for i in range(n):
+            assert O.ring_visit_chunk(i, s, n, -1) == holding[i], "ppermute direction"
+    # Home chunk of an incremental query block, and the page's chunk-start rule.
+    qcs = g["cache_idx_chunk_start"]["query_chunk_size"]
+    for ci in (0, 511, 512, 4095, 4096, 261632):
+        assert O.query_home_chunk(ci, 4096) * 4096 <= ci < (O.query_home_chunk(ci, 4096) + 1) * 4096
+        if ci % qcs == 0:
+            assert (ci // qcs) * qcs == ci
+
+
+ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
+            pin_block_step, pin_lse_merge, pin_schedule]

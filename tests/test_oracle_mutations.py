@@ -1,0 +1,64 @@
+"""Plant plausible mistakes in a copy of the oracle; some pin must catch each.
+
+Each mutation rewrites one expression of ``oracle/attention.py`` (a dropped
+term, a wrong sign or index, a swapped operand), loads the result as a fresh
+module on the CPU and runs the pins against it.  The real oracle is not
+touched.
+"""
+import importlib.util
+import os
+import sys
+import types
+
+import pytest
+
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
+                   "attention.py")
+
+MUTATIONS = [
+    ("gqa head index", "return h_q // (Hq // Hkv)", "return h_q % Hkv"),
+    ("strict causal", "return k_pos[None, :] <= q_pos[:, None]", "return k_pos[None, :] < q_pos[:, None]"),
+    ("reversed causal", "return k_pos[None, :] <= q_pos[:, None]", "return k_pos[None, :] >= q_pos[:, None]"),
+    ("cache_idx ignored", "base = 0 if cache_idx < 0 else int(cache_idx)", "base = 0"),
+    ("scale dropped", "s = scale * (q[b, r, h, :] @ k[b, :n_keys, hk, :].T)", "s = (q[b, r, h, :] @ k[b, :n_keys, hk, :].T)"),
+    ("no normalisation", "o[has] = (w[has] @ v[b, :n_keys, hk, :]) / l[has, None]", "o[has] = (w[has] @ v[b, :n_keys, hk, :])"),
+    ("k used as v", "o[has] = (w[has] @ v[b, :n_keys, hk, :]) / l[has, None]", "o[has] = (w[has] @ k[b, :n_keys, hk, :]) / l[has, None]"),
+    ("lse drops max", "has, m + np.log(np.where(has, l, 1.0)), NEG_INF)", "has, np.log(np.where(has, l, 1.0)), NEG_INF)"),
+    ("rescale of l dropped", "l[b, h] = alpha * l[b, h] + p.sum(axis=1)", "l[b, h] = l[b, h] + p.sum(axis=1)"),
+    ("rescale of acc dropped", "acc[b, h] = alpha[:, None] * acc[b, h] + p @ vc[b, :, hk, :]", "acc[b, h] = acc[b, h] + p @ vc[b, :, hk, :]"),
+    ("rescale sign", "alpha = np.exp(m[b, h] - base)", "alpha = np.exp(base - m[b, h])"),
+    ("block k offset dropped", "k_off + np.arange(Lk, dtype=np.int64)", "np.arange(Lk, dtype=np.int64)"),
+    ("block q offset dropped", "_visible(q_off + np.arange(Lq", "_visible(np.arange(Lq"),
+    ("block scale dropped", "s = scale * (q[b, :, h, :] @ kc[b, :, hk, :].T)", "s = (q[b, :, h, :] @ kc[b, :, hk, :].T)"),
+    ("finalize lse drops m", "lse = np.where(has, m + np.log(safe), NEG_INF)", "lse = np.where(has, np.log(safe), NEG_INF)"),
+    ("ring direction ignored", "return (i + direction * s) % P", "return (i + s) % P"),
+    ("ring always forward from 0", "return (i + direction * s) % P", "return s % P"),
+    ("merge weight sign", "w = np.exp(L - base[None])", "w = np.exp(base[None] - L)"),
+    ("merge lse drops max", "lse = np.where(has, base + np.log(safe), NEG_INF)", "lse = np.where(has, np.log(safe), NEG_INF)"),
+    ("merge unweighted", "out = (w_t * o).sum(axis=0) /", "out = o.sum(axis=0) /"),
+    ("softmax base", "w = np.exp(s - base[:, None])", "w = np.exp(s - base[:, None] - 1.0)"),
+]
+
+
+def _load_mutant(old, new):
+    text = open(SRC).read()
+    assert text.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    text = text.replace(old, new)
+    mod = types.ModuleType("oracle_mutant")
+    mod.__file__ = SRC
+    exec(compile(text, SRC + ":mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_mutation_is_caught(name, old, new):
+    mutant = _load_mutant(old, new)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(mutant)
+        except Exception as e:  # AssertionError or numerical breakage
+            caught.append(f"{pin.__name__}: {type(e).__name__}")
+    assert caught, f"mutation '{name}' passed every pin"

@@ -1,0 +1,111 @@
+"""Seeded synthetic inputs for exact blockwise (ring) attention.
+
+This module is shared by the CUDA path's tests/bench and by the CPU oracle's
+tests.  It holds shapes and random-number recipes only: no attention
+arithmetic lives here, so neither side can borrow the other's math through it.
+
+Every tensor is drawn as float32 standard normal from a seeded
+``torch.Generator`` on the requested device, optionally multiplied by an exact
+power of two, then cast (round-to-nearest-even) to the workload's dtype.  The
+oracle always consumes the *cast* values, upcast to float64, so both sides see
+bit-identical inputs.
+
+Layouts (token-major, row-major contiguous):
+  q, out : [B, N_q,  Hq,  d]
+  k, v   : [B, N_kv, Hkv, d]
+  lse    : [B, Hq, N_q]   (float32, natural log)
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+__all__ = ["Workload", "CONFIGS", "make_qkv", "workload", "small"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, ring split and the input recipe."""
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N_q: int
+    N_kv: int
+    d: int
+    dtype: str            # "bf16" or "f32": element type of q/k/v/out
+    causal: bool
+    P: int                # number of virtual ring chunks the KV sequence is cut into
+    chunk: int            # tokens per chunk; N_kv == P * chunk
+    cache_idx: int = -1   # -1: plain prefill (N_q == N_kv); >= 0: queries sit at cache_idx + t
+    k_scale: float = 1.0  # exact power-of-two multiplier applied to K before the cast
+    seed: int = 0         # q uses seed, k seed+1, v seed+2
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(self.d) ** 0.5
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return {"bf16": torch.bfloat16, "f32": torch.float32}[self.dtype]
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five problems the hot path is specified on, plus decode-shaped variants of
+# the incremental-query case (same KV cache, 1 or 8 new tokens).
+CONFIGS = {
+    1: Workload("tiny_exact_f32_N1024", B=1, Hq=1, Hkv=1, N_q=1024, N_kv=1024, d=64,
+                dtype="f32", causal=False, P=4, chunk=256, seed=1000),
+    2: Workload("llama7b_prefill_N32768", B=1, Hq=32, Hkv=32, N_q=32768, N_kv=32768, d=128,
+                dtype="bf16", causal=True, P=8, chunk=4096, seed=2000),
+    3: Workload("gqa_prefill_N131072", B=1, Hq=32, Hkv=8, N_q=131072, N_kv=131072, d=128,
+                dtype="bf16", causal=True, P=16, chunk=8192, k_scale=2.0, seed=3000),
+    4: Workload("prefill_N1048576", B=1, Hq=8, Hkv=1, N_q=1048576, N_kv=1048576, d=128,
+                dtype="bf16", causal=True, P=64, chunk=16384, seed=4000),
+    5: Workload("cache_idx_query_Nq512_Nkv262144", B=4, Hq=32, Hkv=8, N_q=512, N_kv=262144, d=128,
+                dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 512, seed=5000),
+    "5d1": Workload("cache_idx_decode_Nq1_Nkv262144", B=4, Hq=32, Hkv=8, N_q=1, N_kv=262144, d=128,
+                    dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 1, seed=5100),
+    "5d8": Workload("cache_idx_decode_Nq8_Nkv262144", B=4, Hq=32, Hkv=8, N_q=8, N_kv=262144, d=128,
+                    dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5200),
+}
+
+
+def workload(key) -> Workload:
+    return CONFIGS[key]
+
+
+def small(B=1, Hq=2, Hkv=1, N_q=200, N_kv=None, d=64, dtype="bf16", causal=True, P=2,
+          chunk=None, cache_idx=-1, k_scale=1.0, seed=7, name="small") -> Workload:
+    """A small problem for parity tests (sizes the CPU oracle finishes quickly)."""
+    if N_kv is None:
+        N_kv = N_q if cache_idx < 0 else cache_idx + N_q
+    if chunk is None:
+        chunk = N_kv // P
+    return Workload(name, B=B, Hq=Hq, Hkv=Hkv, N_q=N_q, N_kv=N_kv, d=d, dtype=dtype,
+                    causal=causal, P=P, chunk=chunk, cache_idx=cache_idx, k_scale=k_scale,
+                    seed=seed)
+
+
+def _randn(shape, seed: int, device, mult: float, dtype: torch.dtype) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if mult != 1.0:
+        x.mul_(mult)          # power of two: exact in float32
+    return x.to(dtype)
+
+
+def make_qkv(w: Workload, device="cpu", seed: Optional[int] = None):
+    """Return (q, k, v) for workload ``w`` on ``device`` in ``w``'s dtype."""
+    s = w.seed if seed is None else seed
+    dt = w.torch_dtype
+    q = _randn((w.B, w.N_q, w.Hq, w.d), s + 0, device, 1.0, dt)
+    k = _randn((w.B, w.N_kv, w.Hkv, w.d), s + 1, device, w.k_scale, dt)
+    v = _randn((w.B, w.N_kv, w.Hkv, w.d), s + 2, device, 1.0, dt)
+    return q, k, v
