@@ -1,0 +1,398 @@
+"""Benchmark of the exact blockwise (ring) attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+One step = one forward pass of the whole path (ring_attn_fwd through the C
+ABI) over one batch of synthetic inputs already resident in HBM.  The
+default workload is the Llama-7B-like causal prefill (B=1, Hq=Hkv=32,
+d=128, N=32768, bf16, P=8 chunks of 4096).  With --gpus N > 1 (launched by
+torch.distributed.run) every rank runs its own seeded copy of the workload
+(data-parallel replicas, weak scaling, no collective on the data path);
+the timed region is bracketed by barriers and its duration is the maximum
+over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU float64 oracle on this host's cores on a
+bounded sample of the same workload (the reference arm; there is no
+reference GPU implementation).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
+# kernel, from ncu captures (profiles/), keyed by workload, with the hash of
+# the kernel sources they were taken on.  A stale hash reports null.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_exact_blockwise_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_key(s: str):
+    return int(s) if s.isdigit() else s
+
+
+def flops_of(w: workloads.Workload) -> float:
+    """Algorithmic FLOPs: 4*d per visible (query, key) pair (QK^T and PV).
+
+    Causal prefill counts half of the square (2*B*Hq*N^2*d); an incremental
+    query block counts its exact visible pairs."""
+    if w.cache_idx < 0:
+        pairs = w.N_q * w.N_kv * (0.5 if w.causal else 1.0)
+    elif w.causal:
+        pairs = w.N_q * (w.cache_idx + 1) + w.N_q * (w.N_q - 1) / 2.0
+    else:
+        pairs = float(w.N_q * w.N_kv)
+    return 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def hbm_bytes_of(w: workloads.Workload) -> float:
+    """Minimum HBM traffic: q, k, v read once, out written once, lse written."""
+    es = 2 if w.dtype == "bf16" else 4
+    return es * (2 * w.B * w.N_q * w.Hq * w.d + 2 * w.B * w.N_kv * w.Hkv * w.d) + 4 * w.B * w.Hq * w.N_q
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons via NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self.h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": float(self.max_mhz) if self.max_mhz else None,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ our path
+def run_ours(args, w, rank, world, device):
+    import long_context_exact_blockwise_b200.ringattn as R
+
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    q, k, v = workloads.make_qkv(w, device=device, seed=w.seed + 7919 * rank)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N_q), device=device, dtype=torch.float32)
+    ci = None if w.cache_idx < 0 else w.cache_idx
+    fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
+
+    def step():
+        fn(q, k, v, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
+           stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if R.ring_attn_sync_status(stream) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    clocks = ClockSampler(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(device)
+    launches0 = R.ring_attn_launch_count()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    barrier()
+    launches = R.ring_attn_launch_count() - launches0
+    ms_total = t0.elapsed_time(t1)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = R.ring_attn_sync_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status word {status} after the timed region")
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    hq = q.cpu().pin_memory()
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        fn(dq, dk, dv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
+           stream=stream)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+    res = dict(ms_total=ms_total, per_launch_ms=per_launch, launches=launches, clocks=clocks.summary(),
+               e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, host_inputs=(hq, hk, hv))
+    return res
+
+
+# ------------------------------------------------------------ CPU oracle legs
+def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
+    """Time the float64 oracle on random (row, head) samples of workload w
+    until about budget_s seconds of CPU work are done.  Returns
+    (flops_done, seconds, rows_done, threads)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+    except Exception:  # pragma: no cover
+        threadpool_info = None
+    q, k, v = host_qkv
+    rng = np.random.default_rng(seed)
+    G = w.Hq // w.Hkv
+    kf = {}
+    flops = 0.0
+    rows_done = 0
+    t_start = time.perf_counter()
+    elapsed = 0.0
+    while elapsed < budget_s and rows_done < w.N_q * w.Hq:
+        h = int(rng.integers(0, w.Hq))
+        hk = h // G
+        if hk not in kf:
+            kf[hk] = (k[:, :, hk:hk + 1].double().numpy(), v[:, :, hk:hk + 1].double().numpy())
+        r0 = int(rng.integers(0, max(1, w.N_q - 16)))
+        nr = min(16, w.N_q - r0)
+        qs = q[:, r0:r0 + nr, h:h + 1].double().numpy()
+        base = (0 if w.cache_idx < 0 else w.cache_idx) + r0
+        t0 = time.perf_counter()
+        oracle.attention_ref(qs, kf[hk][0], kf[hk][1], causal=w.causal, scale=w.scale, cache_idx=base)
+        elapsed += time.perf_counter() - t0
+        vis = [(base + i + 1) if w.causal else w.N_kv for i in range(nr)]
+        flops += 4.0 * w.d * w.B * sum(min(x, w.N_kv) for x in vis)
+        rows_done += nr
+        if time.perf_counter() - t_start > 4 * budget_s:
+            break
+    threads = os.cpu_count()
+    if threadpool_info is not None:
+        info = threadpool_info()
+        if info:
+            threads = max(int(x.get("num_threads", 1)) for x in info)
+    return flops, elapsed, rows_done, threads
+
+
+def host_inputs(w):
+    return workloads.make_qkv(w, device="cpu")
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="2", help="workload key: 1..5, 5d1, 5d8 (default 2)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    w = workloads.CONFIGS[config_key(args.config)]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    peaks, peak_src = load_peaks()
+    flops = flops_of(w)
+    config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
+              "causal": w.causal, "P": w.P, "chunk": w.chunk, "cache_idx": w.cache_idx, "k_scale": w.k_scale,
+              "global_batch": w.B * world, "l2": "inputs larger than the 126 MB L2, no flush"
+              if hbm_bytes_of(w) > 126e6 else "inputs fit in L2 (small correctness case)",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        hq = host_inputs(w)
+        budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+        for _ in range(args.warmup):
+            oracle_sample(w, hq, budget / 4)
+        tot_f, tot_s, tot_rows, threads = 0.0, 0.0, 0, 1
+        for i in range(args.steps):
+            f_, s_, r_, threads = oracle_sample(w, hq, budget, seed=i + 1)
+            tot_f += f_
+            tot_s += s_
+            tot_rows += r_
+        val = tot_f / tot_s / 1e12
+        line = {"impl": "reference", "metric": "attention fwd TFLOP/s", "value": val, "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * flops / (val * 1e12), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                 "sample": f"{tot_rows} random (row, head) query rows in runs of 16, "
+                                           f"{tot_s:.1f} s of float64 oracle work over {args.steps} steps"},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    device = local_rank
+    res = run_ours(args, w, rank, world, device)
+    ms_step = res["ms_total"] / args.steps
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    launch_ms = statistics.mean(res["per_launch_ms"])
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    bound = "tensor"
+    unit = "TFLOP/s"
+    if w.dtype == "f32":
+        bound, unit = "alu", "TFLOP/s"
+        # FP32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock.
+        peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+    elif w.cache_idx >= 0 and w.N_q * (w.Hq // w.Hkv) <= 64:
+        bound, unit = "hbm", "GB/s"
+        achieved = hbm_bytes_of(w) / (launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+    src_hash = kernel_source_hash()
+    tr = NCU_TRAFFIC.get(w.name)
+    traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        f_, s_, r_, threads = oracle_sample(w, tuple(x.cpu() for x in res["host_inputs"]), args.cpu_budget)
+        cpu = {"value": f_ / s_ / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{r_} random (row, head) query rows in runs of 16 of this workload, {s_:.1f} s of "
+                         f"float64 oracle work on the host"}
+    e2e_val = flops * world / (res["e2e_ms"] * 1e-3) / 1e12
+    line = {
+        "metric": "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config,
+        "tokens_per_s": w.B * w.N_q * world / (ms_step * 1e-3),
+        "hbm_gbs_algorithmic": hbm_bytes_of(w) * world / (ms_step * 1e-3) / 1e9,
+        "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} ({'burst' if bound == 'tensor' else bound})",
+                     "kernel": "fwd_sm100_kernel" if w.dtype == "bf16" else "simt_attn_kernel",
+                     "algorithmic_per_launch": flops if unit == "TFLOP/s" else hbm_bytes_of(w)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * ring_attn.h -- C ABI of the exact blockwise (ring) attention library for
+ * NVIDIA B200 (sm_100a).  Shared object: libringattn.so.
+ *
+ * The operation (attention definition on "Billion-token context window
+ * engineering", core-challenge paragraph, and "Ring Attention: the secret of
+ * million-token context" §2.3): for every batch b, query head h and query
+ * row t,
+ *     out[b,t,h,:] = sum_j softmax_j(scale * q[b,t,h,:] . k[b,j,hk,:]) v[b,j,hk,:]
+ *     lse[b,h,t]   = ln sum_j exp(scale * q[b,t,h,:] . k[b,j,hk,:])
+ * over the keys j visible to row t, computed blockwise: the KV sequence is
+ * cut into P chunks ("Ring Attention..." §2.1) and each query chunk i visits
+ * KV chunk (i+s) mod P at step s (§2.2 figure), folding each visit into
+ * running (max, sum, output) statistics (§3.1 two-level loop) that are
+ * normalised once over all keys ("From hundreds of milliseconds to a million
+ * tokens", system layer 4: global softmax normalisation).
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are row-major and contiguous, token-major:
+ *       q, out        [B, N_q,  Hq,  d]
+ *       k, v          [B, N_kv, Hkv, d]
+ *       lse           [B, Hq, N_q]           float32, natural log
+ *       acc           [B, Hq, Lq, d]         float32 running numerator
+ *       m, l          [B, Hq, Lq]            float32 running max / sum
+ *       o_parts       [S, B, N_q, Hq, d]     float32, each part normalised
+ *       lse_parts     [S, B, Hq, N_q]        float32
+ *   - GQA: query head h reads KV head h / (Hq / Hkv); Hq % Hkv == 0.
+ *   - Causal masking is per token: key position p_k is visible to query
+ *     position p_q iff p_k <= p_q ("RingAttention inference: using
+ *     cache_idx", basic configuration: causal_block_size = 1).
+ *   - d must be 64 or 128.  bf16 entry points need every pointer 16-byte
+ *     aligned (the tensor-memory-access unit reads them).
+ *   - Every pointer named q, k, v, out, lse, acc, m, l, o_parts, lse_parts
+ *     is DEVICE memory owned by the caller; the library keeps no reference
+ *     after the call returns and frees nothing it did not allocate.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work
+ *     is enqueued asynchronously on it; no call synchronises unless the
+ *     environment variable RINGATTN_DEBUG=1 is set (then each call
+ *     synchronises and also reports the device status word).
+ *   - Every call returns a ring_attn_status.  Arguments are validated on the
+ *     host before anything is launched; an invalid call launches nothing.
+ *     ring_attn_error_string() turns a status into text; after
+ *     RA_ERR_CUDA, ring_attn_last_error() holds the CUDA message.
+ *   - A row with no visible key (possible only through block_step or
+ *     lse_merge inputs that cover no key for it) gives out = 0, lse = -inf.
+ */
+#ifndef RING_ATTN_H_
+#define RING_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad d, Hq % Hkv != 0, N_kv != P*chunk, ... */
+  RA_ERR_UNSUPPORTED = 2,    /* the current device is not sm_100 */
+  RA_ERR_CUDA = 3,           /* a CUDA call or kernel launch failed; see ring_attn_last_error() */
+  RA_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait expired; its outputs are undefined */
+  RA_ERR_OOM = 5             /* stream-ordered workspace allocation failed */
+} ring_attn_status;
+
+#define RA_DTYPE_BF16 0
+#define RA_DTYPE_F32 1
+
+/*
+ * ring_attn_fwd -- full forward pass, bf16 q/k/v/out, float32 lse.
+ *
+ * The sequence of N_kv keys is cut into P chunks of `chunk` tokens
+ * ("Ring Attention..." §2.1); N_kv == P * chunk is required (a length that is
+ * not a multiple of P is rejected, the pitfall listed in "RingAttention and
+ * RAG compared", §2.3).
+ *   cache_idx == -1: prefill.  N_q == N_kv; query row t sits at position t
+ *       and belongs to query chunk i = t / chunk, which visits KV chunk
+ *       (i+s) mod P at step s.
+ *   cache_idx >= 0: incremental query ("RingAttention inference: using
+ *       cache_idx", how cache_idx works).  Query row t sits at position
+ *       cache_idx + t; cache_idx + N_q <= N_kv is required; the block of
+ *       queries is homed at chunk cache_idx / chunk.  The KV cache holds the
+ *       new tokens' own keys.  This path splits the KV range over several
+ *       CTAs and merges their partials (a stream-ordered workspace of
+ *       about S*B*N_q*Hq*(d+1)*4 bytes is allocated and freed on `stream`).
+ * scale multiplies q.k (1/sqrt(d) for standard attention).  The result does
+ * not depend on P or chunk except through rounding.
+ * Returns RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA or
+ * RA_ERR_OOM.
+ */
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                  int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
+                  int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                  void* stream);
+
+/*
+ * ring_attn_fwd_f32 -- the same operation with float32 q/k/v/out, computed
+ * in float32 on CUDA cores (no TF32 tensor cores: the float32 path is held
+ * to 1e-4 absolute error).  Same arguments, conventions and statuses.
+ */
+int ring_attn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse,
+                      int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
+                      int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                      void* stream);
+
+/*
+ * ring_attn_block_step -- one ring visit ("Ring Attention..." §3.1: the
+ * flash-attention call on one received KV chunk).  Folds the attention of
+ * q_chunk [B, Lq, Hq, d] (global positions q_off + t) against
+ * k_chunk/v_chunk [B, Lk, Hkv, d] (global positions k_off + j) into the
+ * caller's running state, in place:
+ *     m'   = max(m, max_j s_j)             s_j = scale * q . k_j (masked: -inf)
+ *     l'   = exp(m - m') l + sum_j exp(s_j - m')
+ *     acc' = exp(m - m') acc + sum_j exp(s_j - m') v_j
+ * m is in natural-log units.  The empty state is acc = 0, m = -inf, l = 0;
+ * a visit whose keys are all masked leaves a row unchanged.
+ * dtype selects the element type of q/k/v chunks: RA_DTYPE_BF16 or
+ * RA_DTYPE_F32.  acc/m/l are always float32 and are read and written.
+ */
+int ring_attn_block_step(const void* q_chunk, const void* k_chunk, const void* v_chunk,
+                         int64_t q_off, int64_t k_off, float* acc, float* m, float* l,
+                         int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d,
+                         int causal, float scale, int dtype, void* stream);
+
+/*
+ * ring_attn_finalize -- out = acc / l, lse = m + ln l (rows with l == 0 give
+ * out = 0, lse = -inf).  acc [B, Hq, Lq, d], m/l [B, Hq, Lq] in; out
+ * [B, Lq, Hq, d] of type out_dtype (RA_DTYPE_BF16 or RA_DTYPE_F32) and lse
+ * [B, Hq, Lq] out.  This is the global normalisation step of "From hundreds
+ * of milliseconds to a million tokens", system layer 4.
+ */
+int ring_attn_finalize(const float* acc, const float* m, const float* l, void* out, float* lse,
+                       int B, int Hq, int64_t Lq, int d, int out_dtype, void* stream);
+
+/*
+ * lse_merge -- merge S normalised partial results by their log-sum-exp
+ * weights (the same global normalisation, applied to partials that each
+ * cover a disjoint key range):
+ *     M = max_s lse_s,  w_s = exp(lse_s - M),  lse = M + ln sum_s w_s,
+ *     out = sum_s w_s O_s / sum_s w_s
+ * o_parts [S, B, N_q, Hq, d] float32, lse_parts [S, B, Hq, N_q] float32 in;
+ * out [B, N_q, Hq, d] (out_dtype) and lse [B, Hq, N_q] out.  A partial with
+ * lse = -inf carries no weight; a row whose partials are all -inf gives
+ * out = 0, lse = -inf.  S >= 1.
+ */
+int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse,
+              int B, int Hq, int64_t N_q, int d, int out_dtype, void* stream);
+
+/*
+ * ring_attn_sync_status -- synchronise `stream`, then read and clear the
+ * device status word that kernels set when a bounded wait expires.  Returns
+ * RA_OK, RA_ERR_DEVICE_TIMEOUT or RA_ERR_CUDA.
+ */
+int ring_attn_sync_status(void* stream);
+
+/* Static description of a status code. Never NULL. */
+const char* ring_attn_error_string(int status);
+
+/* Text of the most recent CUDA failure seen by this thread ("" if none). */
+const char* ring_attn_last_error(void);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int ring_attn_version(void);
+
+/* Number of CUDA kernels this process has launched through the library
+ * (all devices, all threads).  Diagnostic: lets a caller count the launches
+ * inside a timed region. */
+int64_t ring_attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RING_ATTN_H_ */

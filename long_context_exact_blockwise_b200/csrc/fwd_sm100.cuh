@@ -1,0 +1,652 @@
+// Blockwise (ring) attention forward on B200 tensor cores: bf16 inputs,
+// float32 logits and accumulators.
+//
+// What it computes follows "Ring Attention: the secret of million-token
+// context": the KV sequence is cut into P chunks (§2.1); a tile of query
+// rows homed at chunk i visits chunk (i + s) mod P at step s (§2.2 figure);
+// each visit runs the flash-attention inner loop over 128-key tiles held in
+// on-chip memory (§3.1), and the next KV tile is fetched while the current
+// one is computed (§3.2 double buffering, here a TMA ring of smem slots).
+// The partial results are merged by a running max / sum (online softmax)
+// and normalised once over all keys at the end.
+//
+// CTA organisation (one CTA owns NQT query tiles of 128 rows of one head):
+//   warp 0       TMA producer: Q tiles once, then K/V tiles into an
+//                NSLOT-deep ring of shared-memory slots (K_j -> slot 2j,
+//                V_j -> slot 2j+1, modulo NSLOT).
+//   warp 1       MMA issuer (one thread): S_t = Q_t K_j^T into TMEM
+//                (tcgen05.mma, A and B from smem), then O_t += P_t V_j with
+//                P_t read from TMEM.  Q tiles ping-pong: S for one tile is
+//                computed while the other tile's softmax runs.
+//   warp 2       TMEM allocator.
+//   warps 4..    one softmax warpgroup per query tile: thread = query row
+//                (TMEM lane).  Reads S with tcgen05.ld, masks (only tiles
+//                that straddle the causal diagonal or a chunk edge), runs the
+//                exp2 online softmax, writes P (bf16) back over S, rescales O
+//                in TMEM when the row max grew, and writes the epilogue.
+// TMEM columns: S_t at [128 t, 128 t + 128) (P_t aliases its first 64
+// columns), O_t at [128 NQT + D t, ... + D).
+//
+// Every mbarrier wait is bounded (common.cuh); an expired wait sets the
+// device status word and the CTA unwinds without trapping.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+
+#pragma once
+
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ra {
+
+namespace {
+
+constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kTileN = 128;  // keys per KV tile
+
+struct Sm100Params {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  void* out;
+  float* lse;
+  float* o_part;
+  float* lse_part;
+  float* acc;
+  float* m_state;
+  float* l_state;
+  int B, Hq, Hkv, G;
+  long long N_q, N_kv;
+  long long q_pos0, k_pos0;
+  int causal;
+  float scale_log2;
+  long long chunk;
+  int P;
+  int S;
+  int steps_per_split;
+  int n_qblk;
+  int out_f32;
+};
+
+// The sequence of KV tiles one CTA visits: chunks in ring order from `home`,
+// 128-key tiles inside each chunk, keys clipped to [0, lim).
+struct KvCursor {
+  long long chunk, lim;
+  int P, home, s, s_end;
+  long long k0, kend, cend;
+
+  __device__ __forceinline__ void load_chunk() {
+    while (s < s_end) {
+      const int c = (home + s) % P;
+      const long long cb = (long long)c * chunk;
+      const long long ce = min(cb + chunk, lim);
+      if (cb < ce) {
+        k0 = cb;
+        cend = ce;
+        kend = min(k0 + kTileN, cend);
+        return;
+      }
+      ++s;
+    }
+  }
+  __device__ __forceinline__ void init(long long chunk_, long long lim_, int P_, int home_, int s0, int s1) {
+    chunk = chunk_;
+    lim = lim_;
+    P = P_;
+    home = home_;
+    s = s0;
+    s_end = s1;
+    load_chunk();
+  }
+  __device__ __forceinline__ bool valid() const { return s < s_end; }
+  __device__ __forceinline__ void next() {
+    k0 += kTileN;
+    if (k0 < cend) {
+      kend = min(k0 + kTileN, cend);
+    } else {
+      ++s;
+      load_chunk();
+    }
+  }
+};
+
+// Geometry of one query tile of the CTA.
+struct QTile {
+  long long r0;    // first row in the q buffer
+  int nv;          // valid rows (0..128)
+  long long pmin;  // global position of row r0
+  long long pmax;  // global position of the last valid row
+};
+
+template <int D, int NQT, int NSLOT>
+struct Layout {
+  static constexpr int kTileBytes = kTileM * D * 2;  // one bf16 tile of 128 rows x D
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = kQOff + NQT * kTileBytes;
+  static constexpr int kBarOff = kKVOff + NSLOT * kTileBytes;
+  // barriers: q, kv_full[NSLOT], kv_empty[NSLOT], s[NQT], p[NQT], o[NQT], drain
+  static constexpr int kNumBars = 1 + 2 * NSLOT + 3 * NQT + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr uint32_t kTmemCols = (NQT * (128 + D) <= 256) ? 256 : 512;
+  // 1024 bytes of slack for the 1024-byte alignment of the swizzled tiles.  A
+  // CTA that takes all 512 TMEM columns also takes more than half of the
+  // SM's shared memory, so a second CTA never waits on the allocator.
+  static constexpr int kAlloc = (kTmemCols == 512 && kBytes + 1024 < 120 * 1024) ? 120 * 1024 : kBytes + 1024;
+};
+
+__device__ __forceinline__ bool tile_visible(const QTile& q, long long k0, long long k_pos0, int causal) {
+  return q.nv > 0 && (!causal || k_pos0 + k0 <= q.pmax);
+}
+
+__device__ __forceinline__ bool tile_needs_mask(const QTile& q, long long k0, long long kend, long long k_pos0,
+                                                int causal) {
+  return (kend - k0 < kTileN) || (causal && k_pos0 + kend - 1 > q.pmin);
+}
+
+template <int D, int NQT, int NSLOT, int MODE>
+__global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __grid_constant__ Sm100Params p) {
+  using L = Layout<D, NQT, NSLOT>;
+  constexpr int kHalves = D / 64;  // 64-element (128-byte) swizzle columns per tile
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(kTileM, kTileN, 0);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, 1);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto BAR_Q = [&]() { return bar0; };
+  auto BAR_KV_FULL = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto BAR_KV_EMPTY = [&](int i) { return bar0 + 8u * (1 + NSLOT + i); };
+  auto BAR_S = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + t); };
+  auto BAR_P = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + NQT + t); };
+  auto BAR_O = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 2 * NQT + t); };
+  const uint32_t BAR_DRAIN = bar0 + 8u * (1 + 2 * NSLOT + 3 * NQT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (query block, batch, head, split), heaviest blocks first
+  long long x = blockIdx.x;
+  const int sigma = (int)(x % p.S);
+  x /= p.S;
+  const int h = (int)(x % p.Hq);
+  x /= p.Hq;
+  const int b = (int)(x % p.B);
+  x /= p.B;
+  const int qblk = p.n_qblk - 1 - (int)x;
+  const int hk = h / p.G;
+
+  QTile qt[NQT];
+#pragma unroll
+  for (int t = 0; t < NQT; ++t) {
+    qt[t].r0 = (long long)qblk * (NQT * kTileM) + t * kTileM;
+    const long long nv = p.N_q - qt[t].r0;
+    qt[t].nv = (int)(nv < 0 ? 0 : (nv > kTileM ? kTileM : nv));
+    qt[t].pmin = p.q_pos0 + qt[t].r0;
+    qt[t].pmax = qt[t].pmin + (qt[t].nv > 0 ? qt[t].nv - 1 : 0);
+  }
+  // Keys past the block's last query position are invisible to every row.
+  long long last_pos = qt[0].pmax;
+#pragma unroll
+  for (int t = 1; t < NQT; ++t)
+    if (qt[t].nv > 0) last_pos = qt[t].pmax;
+  long long lim = p.N_kv;
+  if (p.causal) lim = min(lim, last_pos - p.k_pos0 + 1);
+  const long long first_rel = qt[0].pmin - p.k_pos0;
+  const int home = first_rel > 0 ? (int)min((long long)(p.P - 1), first_rel / p.chunk) : 0;
+  const int s_begin = sigma * p.steps_per_split;
+  const int s_end = min(p.P, s_begin + p.steps_per_split);
+
+  // ---- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_Q(), 1);
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(BAR_KV_FULL(i), 1);
+      mbar_init(BAR_KV_EMPTY(i), 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(BAR_S(t), 1);
+      mbar_init(BAR_P(t), 128);
+      mbar_init(BAR_O(t), 1);
+    }
+    mbar_init(BAR_DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      prefetch_tmap(&p.tm_q);
+      prefetch_tmap(&p.tm_k);
+      prefetch_tmap(&p.tm_v);
+      uint32_t qbytes = 0;
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (qt[t].nv > 0) qbytes += L::kTileBytes;
+      mbar_arrive_expect_tx(BAR_Q(), qbytes);
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) {
+        if (qt[t].nv == 0) continue;
+#pragma unroll
+        for (int hf = 0; hf < kHalves; ++hf)
+          tma_load_4d(sbase + L::kQOff + t * L::kTileBytes + hf * (kTileM * 128), &p.tm_q, BAR_Q(), hf * 64, h,
+                      (int)qt[t].r0, b);
+      }
+      KvCursor cur;
+      cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+      uint32_t issued = 0;  // slot fills issued (2 per KV tile)
+      bool ok = true;
+      while (ok && cur.valid()) {
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t slot = issued % NSLOT;
+          const uint32_t use = issued / NSLOT;
+          if (!mbar_wait(BAR_KV_EMPTY(slot), (use & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(BAR_KV_FULL(slot), L::kTileBytes);
+          const CUtensorMap* map = kv == 0 ? &p.tm_k : &p.tm_v;
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_4d(sbase + L::kKVOff + slot * L::kTileBytes + hf * (kTileN * 128), map, BAR_KV_FULL(slot),
+                        hf * 64, hk, (int)cur.k0, b);
+          ++issued;
+        }
+        cur.next();
+      }
+      // Let the last fills land before the CTA can exit (normally already
+      // consumed; this matters only when unwinding after a timeout).
+      const uint32_t first = issued > NSLOT ? issued - NSLOT : 0;
+      for (uint32_t f = first; f < issued; ++f) {
+        const uint32_t slot = f % NSLOT;
+        volatile int no_abort = 0;
+        mbar_wait(BAR_KV_FULL(slot), (f / NSLOT) & 1u, &no_abort);
+      }
+      mbar_wait(BAR_Q(), 0, abort_flag);
+    }
+  } else if (warp == 1) {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      bool ok = mbar_wait(BAR_Q(), 0, abort_flag);
+      tc_fence_after();
+      uint64_t qdesc[NQT];
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        qdesc[t] = smem_desc_sw128(sbase + L::kQOff + t * L::kTileBytes, 16, 1024);
+      auto issue_s = [&](int t, uint32_t kslot) {
+        const uint32_t kaddr = sbase + L::kKVOff + kslot * L::kTileBytes;
+        const uint64_t kdesc = smem_desc_sw128(kaddr, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // K-step of 16 elements = 32 bytes inside a 128-byte swizzle row;
+          // every 64 elements move to the next 128-row x 128-byte block.
+          const uint32_t off = (kk / 4) * (kTileM * 128) + (kk % 4) * 32;
+          umma_ss(tmem + 128 * t, qdesc[t] + (off >> 4), kdesc + (off >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR_S(t));
+      };
+      auto issue_pv = [&](int t, uint32_t vslot, bool accumulate_first) {
+        const uint32_t vaddr = sbase + L::kKVOff + vslot * L::kTileBytes;
+        // V tile: keys are rows (128 bytes of d per row and 64-element
+        // column block); for B = V (N = d, K = keys) that is MN-major:
+        // 64-element blocks of d are kTileN*128 bytes apart (LBO), groups of
+        // 8 keys are 1024 bytes apart (SBO).
+        const uint64_t vdesc = smem_desc_sw128(vaddr, kTileN * 128, 1024);
+        const uint32_t o_tmem = tmem + 128 * NQT + D * t;
+        const uint32_t p_tmem = tmem + 128 * t;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk) {
+          // 16 keys per MMA: 2048 bytes of V; 8 TMEM columns of packed P.
+          umma_ts(o_tmem, p_tmem + kk * 8, vdesc + ((kk * 2048) >> 4), kIdescPV,
+                  (accumulate_first || kk > 0) ? 1u : 0u);
+        }
+      };
+      uint32_t p_seen[NQT];
+      bool o_live[NQT];
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) {
+        p_seen[t] = 0;
+        o_live[t] = (MODE == kModeState);
+      }
+      KvCursor cur;
+      cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+      uint32_t j = 0;  // KV tile index
+      if (ok && cur.valid()) {
+        ok = mbar_wait(BAR_KV_FULL(0), 0, abort_flag);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll
+          for (int t = 0; t < NQT; ++t)
+            if (tile_visible(qt[t], cur.k0, p.k_pos0, p.causal)) issue_s(t, 0);
+          tc_commit(BAR_KV_EMPTY(0));
+        }
+      }
+      while (ok && cur.valid()) {
+        KvCursor nxt = cur;
+        nxt.next();
+        const bool has_next = nxt.valid();
+        const uint32_t vfill = 2 * j + 1, kfill = 2 * j + 2;
+        ok = mbar_wait(BAR_KV_FULL(vfill % NSLOT), (vfill / NSLOT) & 1u, abort_flag);
+        tc_fence_after();
+        bool k_ready = false;
+#pragma unroll
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (tile_visible(qt[t], cur.k0, p.k_pos0, p.causal)) {
+            ok = mbar_wait(BAR_P(t), p_seen[t] & 1u, abort_flag);
+            ++p_seen[t];
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, vfill % NSLOT, o_live[t]);
+            o_live[t] = true;
+          }
+          if (has_next && tile_visible(qt[t], nxt.k0, p.k_pos0, p.causal)) {
+            if (!k_ready) {
+              ok = mbar_wait(BAR_KV_FULL(kfill % NSLOT), (kfill / NSLOT) & 1u, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_s(t, kfill % NSLOT);
+          }
+        }
+        if (!ok) break;
+        tc_commit(BAR_KV_EMPTY(vfill % NSLOT));
+        if (has_next) {
+          if (!k_ready) {  // every tile the cursor yields is visible to some query tile
+            ok = mbar_wait(BAR_KV_FULL(kfill % NSLOT), (kfill / NSLOT) & 1u, abort_flag);
+            tc_fence_after();
+          }
+          tc_commit(BAR_KV_EMPTY(kfill % NSLOT));
+        }
+        cur = nxt;
+        ++j;
+      }
+#pragma unroll
+      for (int t = 0; t < NQT; ++t) tc_commit(BAR_O(t));
+      // Drain: all MMAs issued above have completed once this arrives.
+      tc_commit(BAR_DRAIN);
+      volatile int no_abort = 0;
+      mbar_wait(BAR_DRAIN, 0, &no_abort);
+    }
+  } else if (warp >= 4) {
+    // ========================= softmax warpgroups =========================
+    const int t = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int rloc = quad * 32 + lane;  // row inside the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_base + 128 * t;
+    const uint32_t o_tmem = tmem + lane_base + 128 * NQT + D * t;
+    const QTile q = qt[t];
+    const bool row_valid = rloc < q.nv;
+    const long long row = q.r0 + rloc;
+    const long long pos = q.pmin + rloc;
+    const float sl = p.scale_log2;
+
+    float m2 = -INFINITY, l = 0.f, m_in_nat = -INFINITY;
+    if (MODE == kModeState) {
+      // Load the running state: acc into O (TMEM), m (natural log) and l.
+      const long long srow = ((long long)b * p.Hq + h) * p.N_q + (row_valid ? row : 0);
+      if (row_valid) {
+        m_in_nat = p.m_state[srow];
+        m2 = m_in_nat * kLog2e;
+        l = p.l_state[srow];
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          u[i] = row_valid ? __float_as_uint(p.acc[srow * D + c * 32 + i]) : 0u;
+        tmem_st32(o_tmem + c * 32, u);
+      }
+      tc_wait_st();
+    }
+    const float m2_in = m2;
+
+    KvCursor cur;
+    cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+    uint32_t n = 0;
+    bool ok = true;
+    while (cur.valid()) {
+      if (tile_visible(q, cur.k0, p.k_pos0, p.causal)) {
+        if (!mbar_wait(BAR_S(t), n & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float (&r)[32] = *reinterpret_cast<float(*)[32]>(&s[c * 32]);
+          tmem_ld32(s_tmem + c * 32, r);
+        }
+        tc_wait_ld();
+        const bool masked = tile_needs_mask(q, cur.k0, cur.kend, p.k_pos0, p.causal);
+        float mx = -INFINITY;
+        if (masked) {
+          const long long kvis = cur.kend - cur.k0;                       // keys inside chunk and range
+          const long long kcausal = p.causal ? pos - (p.k_pos0 + cur.k0) : (long long)kTileN;  // last visible
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const bool vis = (c < kvis) && (c <= kcausal);
+            s[c] = vis ? s[c] * sl : -INFINITY;
+            mx = fmaxf(mx, s[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            s[c] *= sl;
+            mx = fmaxf(mx, s[c]);
+          }
+        }
+        const float m_new = fmaxf(m2, mx);
+        const float base = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2(m2 - base);
+        float rs = 0.f;
+        // P = exp2(x - base) as bf16 pairs over the first 64 columns of S
+        // (all 128 S columns are already in registers).
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(s[c * 32 + 2 * i] - base);
+            const float p1 = ex2(s[c * 32 + 2 * i + 1] - base);
+            rs += p0 + p1;
+            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+            u[i] = *reinterpret_cast<uint32_t*>(&pk);
+          }
+          tmem_st16(s_tmem + c * 16, u);
+        }
+        l = l * alpha + rs;
+        m2 = m_new;
+        const bool o_has_data = (MODE == kModeState) || n > 0;
+        if (o_has_data && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float r[32];
+            tmem_ld32(o_tmem + c * 32, r);
+            tc_wait_ld();
+            uint32_t u[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(r[i] * alpha);
+            tmem_st32(o_tmem + c * 32, u);
+          }
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR_P(t));
+        ++n;
+      }
+      cur.next();
+    }
+
+    // ------------------------------ epilogue ------------------------------
+    if (ok && n > 0) ok = mbar_wait(BAR_O(t), 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      if (MODE == kModeFinal || MODE == kModeSplit) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const long long ooff = (((long long)(MODE == kModeSplit ? sigma * p.B + b : b) * p.N_q + row) * p.Hq + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float r[32];
+          if (n > 0) {
+            tmem_ld32(o_tmem + c * 32, r);
+            tc_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0.f;
+          }
+          if (!row_valid) continue;
+          if (MODE == kModeSplit || p.out_f32) {
+            float* dst = (MODE == kModeSplit ? p.o_part : static_cast<float*>(p.out)) + ooff + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(r[i] * inv, r[i + 1] * inv, r[i + 2] * inv, r[i + 3] * inv);
+          } else {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + ooff + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 w;
+              __nv_bfloat162 a0 = __floats2bfloat162_rn(r[i] * inv, r[i + 1] * inv);
+              __nv_bfloat162 a1 = __floats2bfloat162_rn(r[i + 2] * inv, r[i + 3] * inv);
+              __nv_bfloat162 a2 = __floats2bfloat162_rn(r[i + 4] * inv, r[i + 5] * inv);
+              __nv_bfloat162 a3 = __floats2bfloat162_rn(r[i + 6] * inv, r[i + 7] * inv);
+              w.x = *reinterpret_cast<uint32_t*>(&a0);
+              w.y = *reinterpret_cast<uint32_t*>(&a1);
+              w.z = *reinterpret_cast<uint32_t*>(&a2);
+              w.w = *reinterpret_cast<uint32_t*>(&a3);
+              *reinterpret_cast<uint4*>(dst + i) = w;
+            }
+          }
+        }
+        if (row_valid) {
+          const float lse_v = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
+          if (MODE == kModeSplit)
+            p.lse_part[(((long long)sigma * p.B + b) * p.Hq + h) * p.N_q + row] = lse_v;
+          else
+            p.lse[((long long)b * p.Hq + h) * p.N_q + row] = lse_v;
+        }
+      } else if (n > 0) {  // kModeState with at least one visible tile
+        const long long srow = ((long long)b * p.Hq + h) * p.N_q + row;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float r[32];
+          tmem_ld32(o_tmem + c * 32, r);
+          tc_wait_ld();
+          if (!row_valid) continue;
+          float* dst = p.acc + srow * D + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+        }
+        if (row_valid) {
+          p.m_state[srow] = (m2 == m2_in) ? m_in_nat : m2 * kLn2;
+          p.l_state[srow] = l;
+        }
+      }
+    }
+  }
+
+  // ---- tear-down: every role has finished (MMAs drained) before TMEM is freed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, L::kTmemCols);
+}
+
+template <int D, int NQT, int NSLOT, int MODE>
+cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) {
+  using L = Layout<D, NQT, NSLOT>;
+  auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE>;
+  static bool attr_set = false;  // per template instance; set once per process
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<(unsigned)grid, 128 + 128 * NQT, L::kAlloc, st>>>(prm);
+  return count_launch(cudaGetLastError());
+}
+
+CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N, int B) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return CUDA_ERROR_NOT_FOUND;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
+  if (a.B <= 0 || a.N_q <= 0) return cudaSuccess;
+  Sm100Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B) != CUDA_SUCCESS ||
+      encode_map(&prm.tm_k, a.k, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS ||
+      encode_map(&prm.tm_v, a.v, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  prm.out = a.out;
+  prm.lse = a.lse;
+  prm.o_part = a.o_part;
+  prm.lse_part = a.lse_part;
+  prm.acc = a.acc;
+  prm.m_state = a.m;
+  prm.l_state = a.l;
+  prm.B = a.B;
+  prm.Hq = a.Hq;
+  prm.Hkv = a.Hkv;
+  prm.G = a.Hq / a.Hkv;
+  prm.N_q = a.N_q;
+  prm.N_kv = a.N_kv;
+  prm.q_pos0 = a.q_pos0;
+  prm.k_pos0 = a.k_pos0;
+  prm.causal = a.causal;
+  prm.scale_log2 = a.scale * kLog2e;
+  prm.chunk = a.chunk;
+  prm.P = a.P;
+  prm.S = mode == kModeSplit ? a.S : 1;
+  prm.steps_per_split = (a.P + prm.S - 1) / prm.S;
+  prm.out_f32 = a.out_f32;
+
+  const bool two = a.N_q > kTileM;  // two query tiles per CTA share each K/V tile
+  const int rows_per_cta = two ? 2 * kTileM : kTileM;
+  prm.n_qblk = (int)((a.N_q + rows_per_cta - 1) / rows_per_cta);
+  const long long grid = (long long)prm.n_qblk * a.B * a.Hq * prm.S;
+  constexpr int NS = 4;
+#define RA_LAUNCH(D_, NQT_)                                                      \
+  switch (mode) {                                                              \
+    case kModeFinal: return launch_cfg<D_, NQT_, NS, kModeFinal>(prm, grid, st); \
+    case kModeSplit: return launch_cfg<D_, NQT_, NS, kModeSplit>(prm, grid, st); \
+    default: return launch_cfg<D_, NQT_, NS, kModeState>(prm, grid, st);        \
+  }
+  if (a.d == 64) {
+    if (two) { RA_LAUNCH(64, 2) } else { RA_LAUNCH(64, 1) }
+  } else {
+    if (two) { RA_LAUNCH(128, 2) } else { RA_LAUNCH(128, 1) }
+  }
+#undef RA_LAUNCH
+}
+
+}  // namespace ra

@@ -1,0 +1,75 @@
+// Host-side launchers of the library's kernels (internal; not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+namespace ra {
+
+// Kernels this process has launched through the library (all devices).
+inline std::atomic<long long>& launch_counter() {
+  static std::atomic<long long> n{0};
+  return n;
+}
+inline cudaError_t count_launch(cudaError_t e) {
+  if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// Output modes of the forward kernels.
+enum FwdMode : int {
+  kModeFinal = 0,  // normalised out (bf16/f32) + lse
+  kModeSplit = 1,  // normalised float32 partial + lse per KV split (merged by lse_merge)
+  kModeState = 2,  // running (acc, m, l) read and written in place (one ring visit)
+};
+
+// One blockwise attention problem as seen by a kernel.  Query row t of the q
+// buffer sits at global position q_pos0 + t; key row j of the k/v buffers at
+// k_pos0 + j.  The k rows are cut into P chunks of `chunk` rows; a tile of
+// query rows homed at chunk i visits chunk (i + s) mod P at step s.
+struct ProblemArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;        // kModeFinal: [B, N_q, Hq, d]
+  float* lse;       // kModeFinal: [B, Hq, N_q]
+  float* o_part;    // kModeSplit: [S, B, N_q, Hq, d]
+  float* lse_part;  // kModeSplit: [S, B, Hq, N_q]
+  float* acc;       // kModeState: [B, Hq, N_q, d]
+  float* m;         // kModeState: [B, Hq, N_q]
+  float* l;         // kModeState: [B, Hq, N_q]
+  int B, Hq, Hkv, d;
+  long long N_q, N_kv;
+  long long q_pos0, k_pos0;
+  int causal;
+  float scale;
+  long long chunk;
+  int P;
+  int S;            // KV splits (kModeSplit), 1 otherwise
+  int out_f32;      // kModeFinal: 1 = float32 out, 0 = bf16 out
+};
+
+// Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.
+cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
+
+// CUDA-core float32 path (also serves float32 block steps).
+cudaError_t launch_fwd_simt_f32(const ProblemArgs& a, int mode, cudaStream_t stream);
+
+// out = acc / l, lse = m + ln l.
+cudaError_t launch_finalize(const float* acc, const float* m, const float* l, void* out, float* lse,
+                            int B, int Hq, long long Lq, int d, int out_f32, cudaStream_t stream);
+
+// Log-sum-exp merge of S normalised partials.
+cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse,
+                             int B, int Hq, long long N_q, int d, int out_f32, cudaStream_t stream);
+
+// Resolve cuTensorMapEncodeTiled through the runtime (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace ra

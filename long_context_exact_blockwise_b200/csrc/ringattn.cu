@@ -1,0 +1,310 @@
+// C ABI of libringattn.so (declared in include/ring_attn.h): argument
+// validation, device checks, dispatch to the kernels, stream-ordered
+// workspace for the split-KV path, and the device status word.
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.h"
+
+// The kernels and their launchers (one translation unit: the status word is
+// shared without relocatable device code).
+#include "fwd_sm100.cuh"
+#include "fwd_simt.cuh"
+#include "merge.cuh"
+
+namespace ra {
+
+namespace {
+
+thread_local std::string t_last_error;
+
+int set_cuda_error(cudaError_t e, const char* where) {
+  t_last_error = std::string(where) + ": " + cudaGetErrorName(e) + ": " + cudaGetErrorString(e);
+  return RA_ERR_CUDA;
+}
+
+bool env_flag(const char* name) {
+  const char* v = std::getenv(name);
+  return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+const char* env_str(const char* name) {
+  const char* v = std::getenv(name);
+  return v ? v : "";
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 1 on sm_100 devices; 0 otherwise; -1 if no device could be queried.
+int device_is_sm100(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (num_sms) *num_sms = sms;
+  return (major == 10 && minor == 0) ? 1 : 0;
+}
+
+int check_device(int* num_sms) {
+  const int r = device_is_sm100(num_sms);
+  if (r == 1) return RA_OK;
+  t_last_error = r < 0 ? "no CUDA device available" : "device is not sm_100 (B200)";
+  return RA_ERR_UNSUPPORTED;
+}
+
+// After a launch: report launch errors; in debug mode also synchronise and
+// read the device status word.
+int finish(cudaError_t e, cudaStream_t st, const char* where) {
+  if (e != cudaSuccess) return set_cuda_error(e, where);
+  if (env_flag("RINGATTN_DEBUG")) {
+    e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return set_cuda_error(e, where);
+    int status = 0;
+    e = cudaMemcpyFromSymbol(&status, g_status, sizeof(int));
+    if (e != cudaSuccess) return set_cuda_error(e, "cudaMemcpyFromSymbol(status)");
+    if (status != 0) {
+      const int zero = 0;
+      cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+      return status;
+    }
+  }
+  return RA_OK;
+}
+
+// Common shape checks for the forward entry points.
+int validate_fwd(const void* q, const void* k, const void* v, const void* out, const void* lse, int B, int Hq,
+                 int Hkv, int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx,
+                 float scale, bool need_align16) {
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (P < 1 || chunk < 1 || N_kv < 1 || N_q < 0) return RA_ERR_INVALID_ARG;
+  if (N_kv / P != chunk || N_kv % P != 0) return RA_ERR_INVALID_ARG;  // N_kv == P * chunk
+  if (N_q > INT32_MAX || N_kv > INT32_MAX) return RA_ERR_INVALID_ARG;
+  if (cache_idx < -1) return RA_ERR_INVALID_ARG;
+  if (cache_idx == -1 && N_q != N_kv) return RA_ERR_INVALID_ARG;
+  if (cache_idx >= 0 && cache_idx + N_q > N_kv) return RA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (need_align16 && !(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out))) return RA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return RA_ERR_INVALID_ARG;
+  return RA_OK;
+}
+
+// Number of KV splits for an incremental query: enough CTAs to keep every SM
+// busy for several waves.  RINGATTN_SPLITS overrides.
+int choose_splits(long long items, int P, int num_sms, long long n_q) {
+  const char* ov = std::getenv("RINGATTN_SPLITS");
+  if (ov && ov[0]) {
+    int s = std::atoi(ov);
+    return s < 1 ? 1 : (s > P ? P : s);
+  }
+  const long long waves = n_q <= 64 ? 8 : 2;  // decode shapes stream KV: want many CTAs in flight
+  long long s = (waves * num_sms + items - 1) / items;
+  if (s < 1) s = 1;
+  if (s > P) s = P;
+  // Whole ring steps per split.
+  const int sps = (int)((P + s - 1) / s);
+  return (P + sps - 1) / sps;
+}
+
+}  // namespace
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace ra
+
+using namespace ra;
+
+extern "C" {
+
+int ring_attn_version(void) { return 100; }
+
+int64_t ring_attn_launch_count(void) { return (int64_t)launch_counter().load(); }
+
+const char* ring_attn_error_string(int status) {
+  switch (status) {
+    case RA_OK: return "ok";
+    case RA_ERR_INVALID_ARG: return "invalid argument";
+    case RA_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+    case RA_ERR_CUDA: return "CUDA error";
+    case RA_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
+    case RA_ERR_OOM: return "workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+const char* ring_attn_last_error(void) { return t_last_error.c_str(); }
+
+int ring_attn_sync_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaStreamSynchronize");
+  int status = 0;
+  e = cudaMemcpyFromSymbol(&status, g_status, sizeof(int));
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaMemcpyFromSymbol(status)");
+  if (status != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return set_cuda_error(e, "cudaMemcpyToSymbol(status)");
+  }
+  return status;
+}
+
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                  int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                  void* stream) {
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N_q == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv;
+  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.k_pos0 = 0;
+  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.S = 1; a.out_f32 = 0;
+
+  if (cache_idx < 0) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd");
+
+  // Incremental query: split the ring steps over S CTAs per query block and
+  // merge the partials by their log-sum-exp weights.
+  const long long rows_per_cta = N_q > 128 ? 256 : 128;
+  const long long items = (long long)B * Hq * ((N_q + rows_per_cta - 1) / rows_per_cta);
+  const int S = choose_splits(items, P, num_sms, N_q);
+  if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd");
+
+  const size_t o_bytes = (size_t)S * B * N_q * Hq * d * sizeof(float);
+  const size_t l_bytes = (size_t)S * B * Hq * N_q * sizeof(float);
+  void* ws = nullptr;
+  if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
+    t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
+    return RA_ERR_OOM;
+  }
+  cudaError_t e = cudaMallocAsync(&ws, o_bytes + l_bytes, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
+    return RA_ERR_OOM;
+  }
+  a.S = S;
+  a.o_part = static_cast<float*>(ws);
+  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
+  e = launch_fwd_sm100(a, kModeSplit, st);
+  if (e == cudaSuccess) e = launch_lse_merge(a.o_part, a.lse_part, S, out, lse, B, Hq, N_q, d, 0, st);
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
+  return finish(e, st, "ring_attn_fwd(split)");
+}
+
+int ring_attn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B, int Hq,
+                      int Hkv, int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx,
+                      float scale, void* stream) {
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, false);
+  if (r != RA_OK) return r;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(out)) & 3u)
+    return RA_ERR_INVALID_ARG;
+  if (B == 0 || N_q == 0) return RA_OK;
+  if ((r = check_device(nullptr)) != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv;
+  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.k_pos0 = 0;
+  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.S = 1; a.out_f32 = 1;
+  return finish(launch_fwd_simt_f32(a, kModeFinal, st), st, "ring_attn_fwd_f32");
+}
+
+int ring_attn_block_step(const void* q_chunk, const void* k_chunk, const void* v_chunk, int64_t q_off,
+                         int64_t k_off, float* acc, float* m, float* l, int B, int Hq, int Hkv, int64_t Lq,
+                         int64_t Lk, int d, int causal, float scale, int dtype, void* stream) {
+  if (!q_chunk || !k_chunk || !v_chunk || !acc || !m || !l) return RA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (Lq < 0 || Lk < 0 || Lq > INT32_MAX || Lk > INT32_MAX) return RA_ERR_INVALID_ARG;
+  if (q_off < 0 || k_off < 0) return RA_ERR_INVALID_ARG;
+  if (dtype != RA_DTYPE_BF16 && dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (!aligned16(acc) || (reinterpret_cast<uintptr_t>(m) & 3u) || (reinterpret_cast<uintptr_t>(l) & 3u))
+    return RA_ERR_INVALID_ARG;
+  if (dtype == RA_DTYPE_BF16 && !(aligned16(q_chunk) && aligned16(k_chunk) && aligned16(v_chunk)))
+    return RA_ERR_INVALID_ARG;
+  if (B == 0 || Lq == 0 || Lk == 0) return RA_OK;
+  int r = check_device(nullptr);
+  if (r != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q_chunk; a.k = k_chunk; a.v = v_chunk;
+  a.acc = acc; a.m = m; a.l = l;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = Lq; a.N_kv = Lk;
+  a.q_pos0 = q_off; a.k_pos0 = k_off;
+  a.causal = causal; a.scale = scale; a.chunk = Lk; a.P = 1; a.S = 1;
+  cudaError_t e = dtype == RA_DTYPE_BF16 ? launch_fwd_sm100(a, kModeState, st) : launch_fwd_simt_f32(a, kModeState, st);
+  return finish(e, st, "ring_attn_block_step");
+}
+
+int ring_attn_finalize(const float* acc, const float* m, const float* l, void* out, float* lse, int B, int Hq,
+                       int64_t Lq, int d, int out_dtype, void* stream) {
+  if (!acc || !m || !l || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Lq < 0 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
+  if (out_dtype != RA_DTYPE_BF16 && out_dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
+  if (!aligned16(acc) || !aligned16(out)) return RA_ERR_INVALID_ARG;
+  if (B == 0 || Lq == 0) return RA_OK;
+  int r = check_device(nullptr);
+  if (r != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return finish(launch_finalize(acc, m, l, out, lse, B, Hq, Lq, d, out_dtype == RA_DTYPE_F32, st), st,
+                "ring_attn_finalize");
+}
+
+int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse, int B, int Hq,
+              int64_t N_q, int d, int out_dtype, void* stream) {
+  if (!o_parts || !lse_parts || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (S < 1 || B < 0 || Hq < 1 || N_q < 0 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
+  if (out_dtype != RA_DTYPE_BF16 && out_dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(out)) return RA_ERR_INVALID_ARG;
+  if (B == 0 || N_q == 0) return RA_OK;
+  int r = check_device(nullptr);
+  if (r != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return finish(launch_lse_merge(o_parts, lse_parts, S, out, lse, B, Hq, N_q, d, out_dtype == RA_DTYPE_F32, st), st,
+                "lse_merge");
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+"""Python binding of libringattn.so (exact blockwise ring attention, B200).
+
+A thin ctypes layer over ``libringattn.so`` (C ABI in ``include/ring_attn.h``).
+Each function here has the name of the C entry point it calls and does only
+argument marshalling: every step of the computation runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.
+
+If the shared object is missing or cannot be loaded, importing this package
+raises ImportError: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "RingAttnError", "lib", "LIB_PATH",
+    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_block_step", "ring_attn_finalize",
+    "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count",
+    "ring_attn", "init_state",
+    "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
+    "RA_ERR_OOM", "RA_DTYPE_BF16", "RA_DTYPE_F32",
+]
+
+RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_DEVICE_TIMEOUT, RA_ERR_OOM = range(6)
+RA_DTYPE_BF16, RA_DTYPE_F32 = 0, 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libringattn.so")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m long_context_exact_blockwise_b200.build_lib` (needs nvcc)")
+    try:
+        return ctypes.CDLL(LIB_PATH)
+    except OSError as e:  # pragma: no cover
+        raise ImportError(f"cannot load {LIB_PATH}: {e}") from e
+
+
+lib = _load()
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_l = ctypes.c_int64
+_f = ctypes.c_float
+
+_SIGS = {
+    "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_block_step": [_p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _i, _p],
+    "ring_attn_finalize": [_p, _p, _p, _p, _p, _i, _i, _l, _i, _i, _p],
+    "lse_merge": [_p, _p, _i, _p, _p, _i, _i, _l, _i, _i, _p],
+    "ring_attn_sync_status": [_p],
+    "ring_attn_error_string": [_i],
+    "ring_attn_last_error": [],
+    "ring_attn_version": [],
+    "ring_attn_launch_count": [],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_char_p if _name in ("ring_attn_error_string", "ring_attn_last_error") else _i
+lib.ring_attn_launch_count.restype = ctypes.c_int64
+
+
+class RingAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.ring_attn_error_string(status).decode()
+        detail = lib.ring_attn_last_error().decode()
+        super().__init__(f"{where}: status {status} ({msg}){': ' + detail if detail else ''}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != RA_OK:
+        raise RingAttnError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def ring_attn_error_string(status: int) -> str:
+    return lib.ring_attn_error_string(status).decode()
+
+
+def ring_attn_version() -> int:
+    return lib.ring_attn_version()
+
+
+def ring_attn_launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(lib.ring_attn_launch_count())
+
+
+def ring_attn_sync_status(stream=None, device=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib.ring_attn_sync_status(_stream(stream, device))
+
+
+def _fwd(fn, dtype, q, k, v, causal, P, chunk, cache_idx, scale, out, lse, stream):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dtype)
+    B, N_q, Hq, d = q.shape
+    _, N_kv, Hkv, dk = k.shape
+    if k.shape != v.shape or dk != d or k.shape[0] != B:
+        raise ValueError("k and v must be [B, N_kv, Hkv, d] matching q")
+    if chunk is None:
+        chunk = N_kv // P if P > 0 else 0
+    ci = -1 if cache_idx is None else int(cache_idx)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N_q), device=q.device, dtype=torch.float32)
+    _need(out, "out", dtype)
+    _need(lse, "lse", torch.float32)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)),
+            int(chunk), int(P), ci, sc, _stream(stream, q.device))
+    _check(st, fn.__name__)
+    return out, lse
+
+
+def ring_attn_fwd(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None, cache_idx=None,
+                  scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """bf16 forward: q [B,N_q,Hq,d], k/v [B,N_kv,Hkv,d] -> (out bf16, lse f32 [B,Hq,N_q])."""
+    return _fwd(lib.ring_attn_fwd, torch.bfloat16, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
+                stream)
+
+
+def ring_attn_fwd_f32(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None, cache_idx=None,
+                      scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """float32 forward (CUDA-core float32 arithmetic); same layouts as ring_attn_fwd."""
+    return _fwd(lib.ring_attn_fwd_f32, torch.float32, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
+                stream)
+
+
+def ring_attn(q, k, v, *, causal: bool, P: int, cache_idx=None, scale=None, stream=None):
+    """Forward pass choosing the entry point by input dtype (bf16 or float32)."""
+    if q.dtype == torch.float32:
+        return ring_attn_fwd_f32(q, k, v, causal=causal, P=P, cache_idx=cache_idx, scale=scale, stream=stream)
+    return ring_attn_fwd(q, k, v, causal=causal, P=P, cache_idx=cache_idx, scale=scale, stream=stream)
+
+
+def init_state(B: int, Hq: int, Lq: int, d: int, device) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Empty running state for ring_attn_block_step: acc = 0, m = -inf, l = 0."""
+    acc = torch.zeros((B, Hq, Lq, d), device=device, dtype=torch.float32)
+    m = torch.full((B, Hq, Lq), float("-inf"), device=device, dtype=torch.float32)
+    l = torch.zeros((B, Hq, Lq), device=device, dtype=torch.float32)
+    return acc, m, l
+
+
+def ring_attn_block_step(q_chunk, k_chunk, v_chunk, q_off: int, k_off: int, acc, m, l, *, causal: bool,
+                         scale: Optional[float] = None, stream=None) -> None:
+    """Fold one ring visit into (acc, m, l) in place; dtype from q_chunk (bf16 or float32)."""
+    dtype = q_chunk.dtype
+    code = {torch.bfloat16: RA_DTYPE_BF16, torch.float32: RA_DTYPE_F32}.get(dtype)
+    if code is None:
+        raise ValueError("q_chunk must be bf16 or float32")
+    for t, n in ((q_chunk, "q_chunk"), (k_chunk, "k_chunk"), (v_chunk, "v_chunk")):
+        _need(t, n, dtype)
+    for t, n in ((acc, "acc"), (m, "m"), (l, "l")):
+        _need(t, n, torch.float32)
+    B, Lq, Hq, d = q_chunk.shape
+    _, Lk, Hkv, _ = k_chunk.shape
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.ring_attn_block_step(_ptr(q_chunk), _ptr(k_chunk), _ptr(v_chunk), int(q_off), int(k_off), _ptr(acc),
+                                  _ptr(m), _ptr(l), B, Hq, Hkv, Lq, Lk, d, int(bool(causal)), sc, code,
+                                  _stream(stream, q_chunk.device))
+    _check(st, "ring_attn_block_step")
+
+
+def ring_attn_finalize(acc, m, l, *, out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+    """(acc [B,Hq,Lq,d], m, l) -> (out [B,Lq,Hq,d] out_dtype, lse [B,Hq,Lq])."""
+    for t, n in ((acc, "acc"), (m, "m"), (l, "l")):
+        _need(t, n, torch.float32)
+    B, Hq, Lq, d = acc.shape
+    if out is None:
+        out = torch.empty((B, Lq, Hq, d), device=acc.device, dtype=out_dtype)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), device=acc.device, dtype=torch.float32)
+    code = RA_DTYPE_F32 if out.dtype == torch.float32 else RA_DTYPE_BF16
+    st = lib.ring_attn_finalize(_ptr(acc), _ptr(m), _ptr(l), _ptr(out), _ptr(lse), B, Hq, Lq, d, code,
+                                _stream(stream, acc.device))
+    _check(st, "ring_attn_finalize")
+    return out, lse
+
+
+def lse_merge(o_parts, lse_parts, *, out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+    """o_parts [S,B,N_q,Hq,d], lse_parts [S,B,Hq,N_q] (float32) -> (out, lse)."""
+    _need(o_parts, "o_parts", torch.float32)
+    _need(lse_parts, "lse_parts", torch.float32)
+    S, B, N_q, Hq, d = o_parts.shape
+    if out is None:
+        out = torch.empty((B, N_q, Hq, d), device=o_parts.device, dtype=out_dtype)
+    if lse is None:
+        lse = torch.empty((B, Hq, N_q), device=o_parts.device, dtype=torch.float32)
+    code = RA_DTYPE_F32 if out.dtype == torch.float32 else RA_DTYPE_BF16
+    st = lib.lse_merge(_ptr(o_parts), _ptr(lse_parts), S, _ptr(out), _ptr(lse), B, Hq, N_q, d, code,
+                       _stream(stream, o_parts.device))
+    _check(st, "lse_merge")
+    return out, lse

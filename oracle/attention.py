@@ -112,8 +112,10 @@ def attention_ref(q, k, v, *, causal: bool, scale: float, cache_idx: int = -1,
     for b in range(B):
         for hi, h in enumerate(heads):
             hk = _kv_head(h, Hq, Hkv)
-            for r0 in range(0, rows.shape[0], _ROW_BLOCK):
-                r = rows[r0:r0 + _ROW_BLOCK]
+            # Bound the dense score block to about 2^25 entries (256 MB).
+            blk = max(1, min(_ROW_BLOCK, (1 << 25) // max(1, N_kv)))
+            for r0 in range(0, rows.shape[0], blk):
+                r = rows[r0:r0 + blk]
                 qp = pos_all[r]
                 # Keys past the last query position carry zero weight under
                 # causal masking; leave them out of the product.
