@@ -41,7 +41,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 12.351685 GB read + 0.402486 GB written.
+    "llama7b_prefill_N32768": {"bytes": 12.754171e9, "src": "72706bf42e83b2b0"},
+}
 
 
 def kernel_source_hash() -> str:
