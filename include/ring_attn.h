@@ -146,6 +146,33 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
               int B, int Hq, int64_t N_q, int d, int out_dtype, void* stream);
 
 /*
+ * ring_attn_fwd_noalloc -- ring_attn_fwd for incremental queries
+ * (cache_idx >= 0) that allocates no device memory.  The pages have no
+ * counterpart; this exists for callers that cannot let a library allocate:
+ * serving stacks whose own pool owns all device memory, and latency-critical
+ * loops where an allocation could fail, fragment that budget or stall.
+ * Same arguments, layouts and result as ring_attn_fwd.  The split-KV
+ * partials go to a fixed 16 MiB device array inside the library instead of a
+ * workspace:
+ *   - every GPU that loads the library holds those 16 MiB until the process
+ *     exits;
+ *   - a call whose partials need more than 16 MiB (about
+ *     S * B * N_q * Hq * (d + 1) * 4 bytes, S chosen as in ring_attn_fwd) is
+ *     rejected with RA_ERR_INVALID_ARG and a message in
+ *     ring_attn_last_error(); cache_idx == -1 is rejected the same way;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture;
+ *   - all calls share the one array and it keeps the last call's contents:
+ *     calls that may overlap on the GPU (different streams, or different
+ *     host threads on the same device) race and must be serialised by the
+ *     caller.
+ */
+int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                          int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
+                          int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                          void* stream);
+
+/*
  * ring_attn_sync_status -- synchronise `stream`, then read and clear the
  * device status word that kernels set when a bounded wait expires.  Returns
  * RA_OK, RA_ERR_DEVICE_TIMEOUT or RA_ERR_CUDA.

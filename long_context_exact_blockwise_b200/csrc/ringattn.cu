@@ -308,3 +308,95 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Allocation-free incremental query (ring_attn_fwd_noalloc).
+//
+// Some callers cannot let a library allocate device memory: serving stacks
+// whose pool allocator owns the whole HBM budget up front, and latency-critical
+// loops where an allocation could fail, fragment that budget or stall on the
+// allocator.  For them the split-KV partials live in a fixed, file-scope device
+// array instead of a stream-ordered workspace.  Every GPU that loads this
+// library reserves the array until the process exits.
+// ----------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char ra_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch_ptr[256] = {};  // device address of the array, per device ordinal
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress once per device (with that device current) and
+// cached.
+int noalloc_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 256) {
+    t_last_error = "ring_attn_fwd_noalloc: device ordinal out of range";
+    return RA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, ra_noalloc_scratch);
+    if (e != cudaSuccess) return set_cuda_error(e, "cudaGetSymbolAddress(ra_noalloc_scratch)");
+    g_noalloc_scratch_ptr[dev] = p;
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                                     int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk,
+                                     int P, int64_t cache_idx, float scale, void* stream) {
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (cache_idx < 0) {
+    t_last_error = "ring_attn_fwd_noalloc serves incremental queries only (cache_idx >= 0)";
+    return RA_ERR_INVALID_ARG;
+  }
+  if (B == 0 || N_q == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv;
+  a.q_pos0 = cache_idx;
+  a.k_pos0 = 0;
+  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.S = 1; a.out_f32 = 0;
+
+  // Same split count as ring_attn_fwd, so both produce the same partials.
+  const long long rows_per_cta = N_q > 128 ? 256 : 128;
+  const long long items = (long long)B * Hq * ((N_q + rows_per_cta - 1) / rows_per_cta);
+  const int S = choose_splits(items, P, num_sms, N_q);
+  if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd_noalloc");
+
+  const size_t o_bytes = (size_t)S * B * N_q * Hq * d * sizeof(float);
+  const size_t l_bytes = (size_t)S * B * Hq * N_q * sizeof(float);
+  if (o_bytes + l_bytes > kNoAllocScratchBytes) {
+    t_last_error = "ring_attn_fwd_noalloc: this call needs " + std::to_string(o_bytes + l_bytes) +
+                   " bytes of split-KV scratch; the static scratch holds " + std::to_string(kNoAllocScratchBytes) +
+                   " bytes (use ring_attn_fwd, or fewer rows B*N_q*Hq)";
+    return RA_ERR_INVALID_ARG;
+  }
+  void* base = nullptr;
+  if ((r = noalloc_scratch_address(&base)) != RA_OK) return r;
+  // Every partial row and lse the merge reads is written by the split kernel
+  // of this same call, so nothing in the scratch needs clearing first.
+  a.S = S;
+  a.o_part = static_cast<float*>(base);
+  a.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + o_bytes);
+  cudaError_t e = launch_fwd_sm100(a, kModeSplit, st);
+  if (e == cudaSuccess) e = launch_lse_merge(a.o_part, a.lse_part, S, out, lse, B, Hq, N_q, d, 0, st);
+  return finish(e, st, "ring_attn_fwd_noalloc");
+}

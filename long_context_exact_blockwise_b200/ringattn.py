@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
-    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_block_step", "ring_attn_finalize",
+    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_block_step", "ring_attn_finalize",
     "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
@@ -53,6 +53,7 @@ _f = ctypes.c_float
 _SIGS = {
     "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_block_step": [_p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _i, _p],
     "ring_attn_finalize": [_p, _p, _p, _p, _p, _i, _i, _l, _i, _i, _p],
     "lse_merge": [_p, _p, _i, _p, _p, _i, _i, _l, _i, _i, _p],
@@ -153,6 +154,17 @@ def ring_attn_fwd_f32(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = N
                       scale: Optional[float] = None, out=None, lse=None, stream=None):
     """float32 forward (CUDA-core float32 arithmetic); same layouts as ring_attn_fwd."""
     return _fwd(lib.ring_attn_fwd_f32, torch.float32, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
+                stream)
+
+
+def ring_attn_fwd_noalloc(q, k, v, *, causal: bool, P: int, cache_idx: int, chunk: Optional[int] = None,
+                          scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """Incremental-query forward that allocates no device memory inside the
+    library (for callers whose memory is owned by their own pool or budget).
+    Split-KV partials use a fixed 16 MiB device array shared by all calls:
+    calls that may overlap on the GPU race, and over-large calls raise.
+    Pass ``out`` and ``lse`` to avoid allocations on the Python side too."""
+    return _fwd(lib.ring_attn_fwd_noalloc, torch.bfloat16, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
                 stream)
 
 
