@@ -45,6 +45,14 @@ namespace ra {
 namespace {
 
 constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
+// The exponent base may trail the running row max by up to this much (log2
+// units) before O is rescaled: P entries stay <= 2^8, far inside bf16 range.
+constexpr float kRescaleSlack = 8.f;
+// Register split of the two-query-tile kernel (384 threads at 168 registers).
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 88;   // warps 0-3: TMA, MMA issue, TMEM allocation
+constexpr int kRegsSoftmax = 208;  // warps 4-11: the two softmax warpgroups
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * kLaunchRegs, "register split exceeds the launch");
 constexpr int kTileN = 128;  // keys per KV tile
 
 struct Sm100Params {
@@ -72,17 +80,18 @@ struct Sm100Params {
 };
 
 // The sequence of KV tiles one CTA visits: chunks in ring order from `home`,
-// 128-key tiles inside each chunk, keys clipped to [0, lim).
+// 128-key tiles inside each chunk, keys clipped to [0, lim).  Indices are
+// k-buffer rows; the host caps buffers well below 2^31 rows, so 32 bits hold
+// every sum formed here.
 struct KvCursor {
-  long long chunk, lim;
-  int P, home, s, s_end;
-  long long k0, kend, cend;
+  int chunk, lim, P, home, s, s_end;
+  int k0, kend, cend;
 
   __device__ __forceinline__ void load_chunk() {
     while (s < s_end) {
       const int c = (home + s) % P;
-      const long long cb = (long long)c * chunk;
-      const long long ce = min(cb + chunk, lim);
+      const int cb = c * chunk;
+      const int ce = min(cb + chunk, lim);
       if (cb < ce) {
         k0 = cb;
         cend = ce;
@@ -92,7 +101,7 @@ struct KvCursor {
       ++s;
     }
   }
-  __device__ __forceinline__ void init(long long chunk_, long long lim_, int P_, int home_, int s0, int s1) {
+  __device__ __forceinline__ void init(int chunk_, int lim_, int P_, int home_, int s0, int s1) {
     chunk = chunk_;
     lim = lim_;
     P = P_;
@@ -113,13 +122,23 @@ struct KvCursor {
   }
 };
 
-// Geometry of one query tile of the CTA.
+// Geometry of one query tile of the CTA.  kmin / kmax: the k-buffer row
+// whose global position equals that of the tile's first / last valid query
+// row, i.e. under causal masking row r0 + i sees keys k <= kmin + i.
+// Clamped to [-2^30, 2^31 - 4096]: beyond either end the answer is the same.
 struct QTile {
-  long long r0;    // first row in the q buffer
-  int nv;          // valid rows (0..128)
-  long long pmin;  // global position of row r0
-  long long pmax;  // global position of the last valid row
+  int r0;    // first row in the q buffer
+  int nv;    // valid rows (0..128)
+  int kmin;
+  int kmax;
 };
+
+constexpr long long kKeyClampLo = -(1ll << 30);
+constexpr long long kKeyClampHi = (1ll << 31) - 4096;
+
+__device__ __forceinline__ int clamp_key(long long x) {
+  return (int)(x < kKeyClampLo ? kKeyClampLo : (x > kKeyClampHi ? kKeyClampHi : x));
+}
 
 template <int D, int NQT, int NSLOT>
 struct Layout {
@@ -138,13 +157,23 @@ struct Layout {
   static constexpr int kAlloc = (kTmemCols == 512 && kBytes + 1024 < 120 * 1024) ? 120 * 1024 : kBytes + 1024;
 };
 
-__device__ __forceinline__ bool tile_visible(const QTile& q, long long k0, long long k_pos0, int causal) {
-  return q.nv > 0 && (!causal || k_pos0 + k0 <= q.pmax);
+template <int NQT>
+__device__ __forceinline__ QTile make_qtile(int qblk, int t, long long N_q, long long qk_delta) {
+  QTile q;
+  q.r0 = qblk * (NQT * kTileM) + t * kTileM;
+  const long long nv = N_q - q.r0;
+  q.nv = (int)(nv < 0 ? 0 : (nv > kTileM ? kTileM : nv));
+  q.kmin = clamp_key(qk_delta + q.r0);
+  q.kmax = clamp_key(qk_delta + q.r0 + (q.nv > 0 ? q.nv - 1 : 0));
+  return q;
 }
 
-__device__ __forceinline__ bool tile_needs_mask(const QTile& q, long long k0, long long kend, long long k_pos0,
-                                                int causal) {
-  return (kend - k0 < kTileN) || (causal && k_pos0 + kend - 1 > q.pmin);
+__device__ __forceinline__ bool tile_visible(const QTile& q, int k0, int causal) {
+  return q.nv > 0 && (!causal || k0 <= q.kmax);
+}
+
+__device__ __forceinline__ bool tile_needs_mask(const QTile& q, int k0, int kend, int causal) {
+  return (kend - k0 < kTileN) || (causal && kend - 1 > q.kmin);
 }
 
 template <int D, int NQT, int NSLOT, int MODE>
@@ -171,34 +200,33 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (query block, batch, head, split), heaviest blocks first
+  // ---- work item.  KV head outermost so that the CTAs resident at one time
+  // share the same K/V in L2; inside it the heaviest query blocks first
+  // (causal work grows with the block index), then the G query heads of the
+  // group and the KV splits.
   long long x = blockIdx.x;
   const int sigma = (int)(x % p.S);
   x /= p.S;
-  const int h = (int)(x % p.Hq);
-  x /= p.Hq;
-  const int b = (int)(x % p.B);
-  x /= p.B;
-  const int qblk = p.n_qblk - 1 - (int)x;
-  const int hk = h / p.G;
+  const int g = (int)(x % p.G);
+  x /= p.G;
+  const int qblk = p.n_qblk - 1 - (int)(x % p.n_qblk);
+  x /= p.n_qblk;
+  const int hk = (int)(x % p.Hkv);
+  const int b = (int)(x / p.Hkv);
+  const int h = hk * p.G + g;
 
   QTile qt[NQT];
 #pragma unroll
-  for (int t = 0; t < NQT; ++t) {
-    qt[t].r0 = (long long)qblk * (NQT * kTileM) + t * kTileM;
-    const long long nv = p.N_q - qt[t].r0;
-    qt[t].nv = (int)(nv < 0 ? 0 : (nv > kTileM ? kTileM : nv));
-    qt[t].pmin = p.q_pos0 + qt[t].r0;
-    qt[t].pmax = qt[t].pmin + (qt[t].nv > 0 ? qt[t].nv - 1 : 0);
-  }
+  const long long qk_delta = p.q_pos0 - p.k_pos0;
+  for (int t = 0; t < NQT; ++t) qt[t] = make_qtile<NQT>(qblk, t, p.N_q, qk_delta);
   // Keys past the block's last query position are invisible to every row.
-  long long last_pos = qt[0].pmax;
+  int kmax_last = qt[0].kmax;
 #pragma unroll
   for (int t = 1; t < NQT; ++t)
-    if (qt[t].nv > 0) last_pos = qt[t].pmax;
-  long long lim = p.N_kv;
-  if (p.causal) lim = min(lim, last_pos - p.k_pos0 + 1);
-  const long long first_rel = qt[0].pmin - p.k_pos0;
+    if (qt[t].nv > 0) kmax_last = qt[t].kmax;
+  int lim = (int)p.N_kv;
+  if (p.causal) lim = max(0, min(lim, kmax_last + 1));
+  const long long first_rel = qk_delta + qt[0].r0;
   const int home = first_rel > 0 ? (int)min((long long)(p.P - 1), first_rel / p.chunk) : 0;
   const int s_begin = sigma * p.steps_per_split;
   const int s_end = min(p.P, s_begin + p.steps_per_split);
@@ -228,6 +256,13 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Two query tiles: registers move from the producer/MMA warpgroup to the
+  // softmax warpgroups at the head of each role's branch.  The block is
+  // launched with kLaunchRegs per thread (checked on the host before
+  // launch): 128 * 88 + 256 * 208 = 384 * 168.
+  if (warp < 4) {
+    if constexpr (NQT == 2) reg_dealloc<kRegsControl>();
+  }
   if (warp == 0) {
     // =========================== TMA producer ===========================
     if (lane == 0) {
@@ -245,10 +280,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 #pragma unroll
         for (int hf = 0; hf < kHalves; ++hf)
           tma_load_4d(sbase + L::kQOff + t * L::kTileBytes + hf * (kTileM * 128), &p.tm_q, BAR_Q(), hf * 64, h,
-                      (int)qt[t].r0, b);
+                      qt[t].r0, b);
       }
       KvCursor cur;
-      cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+      cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t issued = 0;  // slot fills issued (2 per KV tile)
       bool ok = true;
       while (ok && cur.valid()) {
@@ -325,7 +360,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         o_live[t] = (MODE == kModeState);
       }
       KvCursor cur;
-      cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+      cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t j = 0;  // KV tile index
       if (ok && cur.valid()) {
         ok = mbar_wait(BAR_KV_FULL(0), 0, abort_flag);
@@ -333,7 +368,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         if (ok) {
 #pragma unroll
           for (int t = 0; t < NQT; ++t)
-            if (tile_visible(qt[t], cur.k0, p.k_pos0, p.causal)) issue_s(t, 0);
+            if (tile_visible(qt[t], cur.k0, p.causal)) issue_s(t, 0);
           tc_commit(BAR_KV_EMPTY(0));
         }
       }
@@ -347,7 +382,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         bool k_ready = false;
 #pragma unroll
         for (int t = 0; t < NQT && ok; ++t) {
-          if (tile_visible(qt[t], cur.k0, p.k_pos0, p.causal)) {
+          if (tile_visible(qt[t], cur.k0, p.causal)) {
             ok = mbar_wait(BAR_P(t), p_seen[t] & 1u, abort_flag);
             ++p_seen[t];
             if (!ok) break;
@@ -355,7 +390,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
             issue_pv(t, vfill % NSLOT, o_live[t]);
             o_live[t] = true;
           }
-          if (has_next && tile_visible(qt[t], nxt.k0, p.k_pos0, p.causal)) {
+          if (has_next && tile_visible(qt[t], nxt.k0, p.causal)) {
             if (!k_ready) {
               ok = mbar_wait(BAR_KV_FULL(kfill % NSLOT), (kfill / NSLOT) & 1u, abort_flag);
               if (!ok) break;
@@ -386,22 +421,28 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     }
   } else if (warp >= 4) {
     // ========================= softmax warpgroups =========================
+    if constexpr (NQT == 2) reg_alloc<kRegsSoftmax>();
     const int t = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int rloc = quad * 32 + lane;  // row inside the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + 128 * t;
     const uint32_t o_tmem = tmem + lane_base + 128 * NQT + D * t;
-    const QTile q = qt[t];
+    const QTile q = make_qtile<NQT>(qblk, t, p.N_q, p.q_pos0 - p.k_pos0);
     const bool row_valid = rloc < q.nv;
-    const long long row = q.r0 + rloc;
-    const long long pos = q.pmin + rloc;
-    const float sl = p.scale_log2;
+    const long long row = (long long)q.r0 + rloc;
+    // With scale > 0 the row max is taken on raw scores and the scale is
+    // folded into the exponent's FMA; otherwise scores are scaled first.
+    const bool fold = p.scale_log2 > 0.f;
+    const float sl = fold ? p.scale_log2 : 1.f;
 
+    // m2: the base of the exponentials (log2 units); it trails the true row
+    // max by at most kRescaleSlack, so exp2(x - m2) <= 2^kRescaleSlack and O
+    // needs rescaling only when the max jumps past that.  O, l and m2 always
+    // describe the same sum, so the final out and lse are exact.
     float m2 = -INFINITY, l = 0.f, m_in_nat = -INFINITY;
+    const long long srow = ((long long)b * p.Hq + h) * p.N_q + (row_valid ? row : 0);
     if (MODE == kModeState) {
-      // Load the running state: acc into O (TMEM), m (natural log) and l.
-      const long long srow = ((long long)b * p.Hq + h) * p.N_q + (row_valid ? row : 0);
       if (row_valid) {
         m_in_nat = p.m_state[srow];
         m2 = m_in_nat * kLog2e;
@@ -418,13 +459,14 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
       tc_wait_st();
     }
     const float m2_in = m2;
+    float m_true = m2;  // true running max (kept for the state epilogue)
 
     KvCursor cur;
-    cur.init(p.chunk, lim, p.P, home, s_begin, s_end);
+    cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
     uint32_t n = 0;
     bool ok = true;
     while (cur.valid()) {
-      if (tile_visible(q, cur.k0, p.k_pos0, p.causal)) {
+      if (tile_visible(q, cur.k0, p.causal)) {
         if (!mbar_wait(BAR_S(t), n & 1u, abort_flag)) {
           ok = false;
           break;
@@ -437,56 +479,83 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
           tmem_ld32(s_tmem + c * 32, r);
         }
         tc_wait_ld();
-        const bool masked = tile_needs_mask(q, cur.k0, cur.kend, p.k_pos0, p.causal);
-        float mx = -INFINITY;
-        if (masked) {
-          const long long kvis = cur.kend - cur.k0;                       // keys inside chunk and range
-          const long long kcausal = p.causal ? pos - (p.k_pos0 + cur.k0) : (long long)kTileN;  // last visible
+        if (!fold) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const bool vis = (c < kvis) && (c <= kcausal);
-            s[c] = vis ? s[c] * sl : -INFINITY;
-            mx = fmaxf(mx, s[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            s[c] *= sl;
-            mx = fmaxf(mx, s[c]);
-          }
+          for (int c = 0; c < 128; ++c) s[c] *= p.scale_log2;
         }
-        const float m_new = fmaxf(m2, mx);
-        const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2(m2 - base);
-        float rs = 0.f;
-        // P = exp2(x - base) as bf16 pairs over the first 64 columns of S
-        // (all 128 S columns are already in registers).
+        if (tile_needs_mask(q, cur.k0, cur.kend, p.causal)) {
+          const int kvis = cur.kend - cur.k0;  // keys inside the chunk / range
+          // Last key (tile-relative) this row sees under causal masking.
+          const long long kc = p.causal ? (long long)q.kmin + rloc - cur.k0 : (long long)kTileN;
+          const int kcausal = (int)(kc < -1 ? -1 : (kc > kTileN ? kTileN : kc));
+          const int klast = min(kvis - 1, kcausal);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = (c <= klast) ? s[c] : -INFINITY;
+        }
+        // Row max: four independent chains of 3-input max.
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+        }
+        const float m_tile = fmax3(fmaxf(mx0, mx1), mx2, mx3) * sl;  // -inf stays -inf (sl > 0)
+        m_true = fmaxf(m_true, m_tile);
+        float alpha = 1.f;
+        if (m_tile > m2 + kRescaleSlack) {
+          alpha = ex2(m2 - m_tile);  // 0 when m2 = -inf
+          m2 = m_tile;
+          l *= alpha;
+        }
+        const float base = (m2 == -INFINITY) ? 0.f : m2;
+        const float2 sl2 = make_float2(sl, sl);
+        const float2 nb2 = make_float2(-base, -base);
+        float2 sum0 = make_float2(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
+        // P = exp2(sl * s - base) as bf16 pairs over the first 64 columns of S.
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t u[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(s[c * 32 + 2 * i] - base);
-            const float p1 = ex2(s[c * 32 + 2 * i + 1] - base);
-            rs += p0 + p1;
-            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-            u[i] = *reinterpret_cast<uint32_t*>(&pk);
+          for (int i = 0; i < 16; i += 4) {
+            float2 e0 = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), sl2, nb2);
+            float2 e1 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 2], s[c * 32 + 2 * i + 3]), sl2, nb2);
+            float2 e2 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 4], s[c * 32 + 2 * i + 5]), sl2, nb2);
+            float2 e3 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 6], s[c * 32 + 2 * i + 7]), sl2, nb2);
+            e0 = make_float2(ex2(e0.x), ex2(e0.y));
+            e1 = make_float2(ex2(e1.x), ex2(e1.y));
+            e2 = make_float2(ex2(e2.x), ex2(e2.y));
+            e3 = make_float2(ex2(e3.x), ex2(e3.y));
+            sum0 = __fadd2_rn(sum0, e0);
+            sum1 = __fadd2_rn(sum1, e1);
+            sum2 = __fadd2_rn(sum2, e2);
+            sum3 = __fadd2_rn(sum3, e3);
+            u[i] = pack_bf16x2(e0.x, e0.y);
+            u[i + 1] = pack_bf16x2(e1.x, e1.y);
+            u[i + 2] = pack_bf16x2(e2.x, e2.y);
+            u[i + 3] = pack_bf16x2(e3.x, e3.y);
           }
           tmem_st16(s_tmem + c * 16, u);
         }
-        l = l * alpha + rs;
-        m2 = m_new;
+        const float2 sa = __fadd2_rn(__fadd2_rn(sum0, sum1), __fadd2_rn(sum2, sum3));
+        l += sa.x + sa.y;
         const bool o_has_data = (MODE == kModeState) || n > 0;
         if (o_has_data && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float r[32];
-            tmem_ld32(o_tmem + c * 32, r);
+          for (int c = 0; c < D / 32; c += 2) {
+            float r0[32], r1[32];
+            tmem_ld32(o_tmem + c * 32, r0);
+            tmem_ld32(o_tmem + (c + 1) * 32, r1);
             tc_wait_ld();
-            uint32_t u[32];
+            uint32_t u0[32], u1[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(r[i] * alpha);
-            tmem_st32(o_tmem + c * 32, u);
+            for (int i = 0; i < 32; ++i) {
+              u0[i] = __float_as_uint(r0[i] * alpha);
+              u1[i] = __float_as_uint(r1[i] * alpha);
+            }
+            tmem_st32(o_tmem + c * 32, u0);
+            tmem_st32(o_tmem + (c + 1) * 32, u1);
           }
         }
         tc_wait_st();
@@ -525,14 +594,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
               uint4 w;
-              __nv_bfloat162 a0 = __floats2bfloat162_rn(r[i] * inv, r[i + 1] * inv);
-              __nv_bfloat162 a1 = __floats2bfloat162_rn(r[i + 2] * inv, r[i + 3] * inv);
-              __nv_bfloat162 a2 = __floats2bfloat162_rn(r[i + 4] * inv, r[i + 5] * inv);
-              __nv_bfloat162 a3 = __floats2bfloat162_rn(r[i + 6] * inv, r[i + 7] * inv);
-              w.x = *reinterpret_cast<uint32_t*>(&a0);
-              w.y = *reinterpret_cast<uint32_t*>(&a1);
-              w.z = *reinterpret_cast<uint32_t*>(&a2);
-              w.w = *reinterpret_cast<uint32_t*>(&a3);
+              w.x = pack_bf16x2(r[i] * inv, r[i + 1] * inv);
+              w.y = pack_bf16x2(r[i + 2] * inv, r[i + 3] * inv);
+              w.z = pack_bf16x2(r[i + 4] * inv, r[i + 5] * inv);
+              w.w = pack_bf16x2(r[i + 6] * inv, r[i + 7] * inv);
               *reinterpret_cast<uint4*>(dst + i) = w;
             }
           }
@@ -545,7 +610,8 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
             p.lse[((long long)b * p.Hq + h) * p.N_q + row] = lse_v;
         }
       } else if (n > 0) {  // kModeState with at least one visible tile
-        const long long srow = ((long long)b * p.Hq + h) * p.N_q + row;
+        // Hand back the state relative to the true running max.
+        const float fix = (m_true > m2) ? ex2(m2 - m_true) : 1.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float r[32];
@@ -554,11 +620,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
           if (!row_valid) continue;
           float* dst = p.acc + srow * D + c * 32;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + i) = make_float4(r[i] * fix, r[i + 1] * fix, r[i + 2] * fix, r[i + 3] * fix);
         }
         if (row_valid) {
-          p.m_state[srow] = (m2 == m2_in) ? m_in_nat : m2 * kLn2;
-          p.l_state[srow] = l;
+          p.m_state[srow] = (m_true == m2_in) ? m_in_nat : m_true * kLn2;
+          p.l_state[srow] = l * fix;
         }
       }
     }
@@ -575,11 +642,28 @@ template <int D, int NQT, int NSLOT, int MODE>
 cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) {
   using L = Layout<D, NQT, NSLOT>;
   auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE>;
-  static bool attr_set = false;  // per template instance; set once per process
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
+  if constexpr (NQT == 2) {
+    // The in-kernel register split assumes exactly kLaunchRegs per thread.
+    static int regs = -1;
+    if (regs < 0) {
+      cudaFuncAttributes fa;
+      cudaError_t e0 = cudaFuncGetAttributes(&fa, kern);
+      if (e0 != cudaSuccess) return e0;
+      regs = fa.numRegs;
+    }
+    if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  }
+  // The attribute is per device: set it on every device this instance runs on.
+  static unsigned long long attr_set_mask = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(__atomic_load_n(&attr_set_mask, __ATOMIC_ACQUIRE) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
   }
   kern<<<(unsigned)grid, 128 + 128 * NQT, L::kAlloc, st>>>(prm);
   return count_launch(cudaGetLastError());
@@ -634,17 +718,18 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   const int rows_per_cta = two ? 2 * kTileM : kTileM;
   prm.n_qblk = (int)((a.N_q + rows_per_cta - 1) / rows_per_cta);
   const long long grid = (long long)prm.n_qblk * a.B * a.Hq * prm.S;
-  constexpr int NS = 4;
-#define RA_LAUNCH(D_, NQT_)                                                      \
-  switch (mode) {                                                              \
-    case kModeFinal: return launch_cfg<D_, NQT_, NS, kModeFinal>(prm, grid, st); \
-    case kModeSplit: return launch_cfg<D_, NQT_, NS, kModeSplit>(prm, grid, st); \
-    default: return launch_cfg<D_, NQT_, NS, kModeState>(prm, grid, st);        \
+  // K/V ring depth: as many 128-key slots as shared memory allows
+  // (d=128: 2 query tiles + 5 slots = 224 KB; 1 tile + 6 slots).
+#define RA_LAUNCH(D_, NQT_, NS_)                                                  \
+  switch (mode) {                                                               \
+    case kModeFinal: return launch_cfg<D_, NQT_, NS_, kModeFinal>(prm, grid, st); \
+    case kModeSplit: return launch_cfg<D_, NQT_, NS_, kModeSplit>(prm, grid, st); \
+    default: return launch_cfg<D_, NQT_, NS_, kModeState>(prm, grid, st);        \
   }
   if (a.d == 64) {
-    if (two) { RA_LAUNCH(64, 2) } else { RA_LAUNCH(64, 1) }
+    if (two) { RA_LAUNCH(64, 2, 8) } else { RA_LAUNCH(64, 1, 8) }
   } else {
-    if (two) { RA_LAUNCH(128, 2) } else { RA_LAUNCH(128, 1) }
+    if (two) { RA_LAUNCH(128, 2, 5) } else { RA_LAUNCH(128, 1, 6) }
   }
 #undef RA_LAUNCH
 }

@@ -38,6 +38,9 @@ const char* env_str(const char* name) {
   return v ? v : "";
 }
 
+// Longest q or k/v buffer a call accepts (rows); kernels index rows in 32 bits.
+constexpr int64_t kMaxTokens = (int64_t(1) << 31) - 8192;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // 1 on sm_100 devices; 0 otherwise; -1 if no device could be queried.
@@ -94,7 +97,7 @@ int validate_fwd(const void* q, const void* k, const void* v, const void* out, c
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
   if (P < 1 || chunk < 1 || N_kv < 1 || N_q < 0) return RA_ERR_INVALID_ARG;
   if (N_kv / P != chunk || N_kv % P != 0) return RA_ERR_INVALID_ARG;  // N_kv == P * chunk
-  if (N_q > INT32_MAX || N_kv > INT32_MAX) return RA_ERR_INVALID_ARG;
+  if (N_q > kMaxTokens || N_kv > kMaxTokens) return RA_ERR_INVALID_ARG;
   if (cache_idx < -1) return RA_ERR_INVALID_ARG;
   if (cache_idx == -1 && N_q != N_kv) return RA_ERR_INVALID_ARG;
   if (cache_idx >= 0 && cache_idx + N_q > N_kv) return RA_ERR_INVALID_ARG;
@@ -255,7 +258,7 @@ int ring_attn_block_step(const void* q_chunk, const void* k_chunk, const void* v
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
-  if (Lq < 0 || Lk < 0 || Lq > INT32_MAX || Lk > INT32_MAX) return RA_ERR_INVALID_ARG;
+  if (Lq < 0 || Lk < 0 || Lq > kMaxTokens || Lk > kMaxTokens) return RA_ERR_INVALID_ARG;
   if (q_off < 0 || k_off < 0) return RA_ERR_INVALID_ARG;
   if (dtype != RA_DTYPE_BF16 && dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return RA_ERR_INVALID_ARG;
