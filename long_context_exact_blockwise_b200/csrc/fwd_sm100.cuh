@@ -77,6 +77,9 @@ struct Sm100Params {
   int steps_per_split;
   int n_qblk;
   int out_f32;
+  int gpack;   // query heads packed into one tile (1, or G for incremental queries)
+  int gshift;  // log2(gpack)
+  int tpt;     // tokens per tile: 128 / gpack
 };
 
 // The sequence of KV tiles one CTA visits: chunks in ring order from `home`,
@@ -122,12 +125,14 @@ struct KvCursor {
   }
 };
 
-// Geometry of one query tile of the CTA.  kmin / kmax: the k-buffer row
-// whose global position equals that of the tile's first / last valid query
-// row, i.e. under causal masking row r0 + i sees keys k <= kmin + i.
-// Clamped to [-2^30, 2^31 - 4096]: beyond either end the answer is the same.
+// Geometry of one query tile of the CTA.  A tile holds tpt tokens x gpack
+// heads; tile row r is token tok0 + (r >> gshift) of head h + (r & (gpack-1)).
+// kmin / kmax: the k-buffer row whose global position equals that of the
+// tile's first / last valid token, so under causal masking token tok0 + i
+// sees keys k <= kmin + i.  Clamped to [-2^30, 2^31 - 4096]: beyond either
+// end the answer is the same.
 struct QTile {
-  int r0;    // first row in the q buffer
+  int tok0;  // first token in the q buffer
   int nv;    // valid rows (0..128)
   int kmin;
   int kmax;
@@ -158,13 +163,15 @@ struct Layout {
 };
 
 template <int NQT>
-__device__ __forceinline__ QTile make_qtile(int qblk, int t, long long N_q, long long qk_delta) {
+__device__ __forceinline__ QTile make_qtile(int qblk, int t, long long N_q, long long qk_delta, int tpt,
+                                           int gshift) {
   QTile q;
-  q.r0 = qblk * (NQT * kTileM) + t * kTileM;
-  const long long nv = N_q - q.r0;
-  q.nv = (int)(nv < 0 ? 0 : (nv > kTileM ? kTileM : nv));
-  q.kmin = clamp_key(qk_delta + q.r0);
-  q.kmax = clamp_key(qk_delta + q.r0 + (q.nv > 0 ? q.nv - 1 : 0));
+  q.tok0 = qblk * (NQT * tpt) + t * tpt;
+  const long long nt = N_q - q.tok0;
+  const int ntok = (int)(nt < 0 ? 0 : (nt > tpt ? tpt : nt));
+  q.nv = ntok << gshift;
+  q.kmin = clamp_key(qk_delta + q.tok0);
+  q.kmax = clamp_key(qk_delta + q.tok0 + (ntok > 0 ? ntok - 1 : 0));
   return q;
 }
 
@@ -207,8 +214,9 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   long long x = blockIdx.x;
   const int sigma = (int)(x % p.S);
   x /= p.S;
-  const int g = (int)(x % p.G);
-  x /= p.G;
+  const int g_iter = p.gpack > 1 ? 1 : p.G;  // packed tiles hold the whole group
+  const int g = (int)(x % g_iter);
+  x /= g_iter;
   const int qblk = p.n_qblk - 1 - (int)(x % p.n_qblk);
   x /= p.n_qblk;
   const int hk = (int)(x % p.Hkv);
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   QTile qt[NQT];
 #pragma unroll
   const long long qk_delta = p.q_pos0 - p.k_pos0;
-  for (int t = 0; t < NQT; ++t) qt[t] = make_qtile<NQT>(qblk, t, p.N_q, qk_delta);
+  for (int t = 0; t < NQT; ++t) qt[t] = make_qtile<NQT>(qblk, t, p.N_q, qk_delta, p.tpt, p.gshift);
   // Keys past the block's last query position are invisible to every row.
   int kmax_last = qt[0].kmax;
 #pragma unroll
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     if (qt[t].nv > 0) kmax_last = qt[t].kmax;
   int lim = (int)p.N_kv;
   if (p.causal) lim = max(0, min(lim, kmax_last + 1));
-  const long long first_rel = qk_delta + qt[0].r0;
+  const long long first_rel = qk_delta + qt[0].tok0;
   const int home = first_rel > 0 ? (int)min((long long)(p.P - 1), first_rel / p.chunk) : 0;
   const int s_begin = sigma * p.steps_per_split;
   const int s_end = min(p.P, s_begin + p.steps_per_split);
@@ -239,8 +247,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
       mbar_init(BAR_KV_EMPTY(i), 1);
     }
     for (int t = 0; t < NQT; ++t) {
+      // One arrival per thread of the softmax warps that hold valid rows.
+      const int active_warps = min(4, (qt[t].nv + 31) / 32);
       mbar_init(BAR_S(t), 1);
-      mbar_init(BAR_P(t), 128);
+      mbar_init(BAR_P(t), 32 * max(1, active_warps));
       mbar_init(BAR_O(t), 1);
     }
     mbar_init(BAR_DRAIN, 1);
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 #pragma unroll
         for (int hf = 0; hf < kHalves; ++hf)
           tma_load_4d(sbase + L::kQOff + t * L::kTileBytes + hf * (kTileM * 128), &p.tm_q, BAR_Q(), hf * 64, h,
-                      qt[t].r0, b);
+                      qt[t].tok0, b);
       }
       KvCursor cur;
       cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
@@ -428,9 +438,13 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + 128 * t;
     const uint32_t o_tmem = tmem + lane_base + 128 * NQT + D * t;
-    const QTile q = make_qtile<NQT>(qblk, t, p.N_q, p.q_pos0 - p.k_pos0);
+    const QTile q = make_qtile<NQT>(qblk, t, p.N_q, p.q_pos0 - p.k_pos0, p.tpt, p.gshift);
     const bool row_valid = rloc < q.nv;
-    const long long row = (long long)q.r0 + rloc;
+    const int tl = rloc >> p.gshift;                   // token inside the tile
+    const int head = h + (rloc & (p.gpack - 1));       // query head of this row
+    const long long row = (long long)q.tok0 + tl;      // token in the q buffer
+    // Warps whose 32 rows are all empty (short incremental queries) sit out.
+    const bool warp_active = quad * 32 < q.nv;
     // With scale > 0 the row max is taken on raw scores and the scale is
     // folded into the exponent's FMA; otherwise scores are scaled first.
     const bool fold = p.scale_log2 > 0.f;
@@ -441,7 +455,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     // needs rescaling only when the max jumps past that.  O, l and m2 always
     // describe the same sum, so the final out and lse are exact.
     float m2 = -INFINITY, l = 0.f, m_in_nat = -INFINITY;
-    const long long srow = ((long long)b * p.Hq + h) * p.N_q + (row_valid ? row : 0);
+    const long long srow = ((long long)b * p.Hq + head) * p.N_q + (row_valid ? row : 0);
     if (MODE == kModeState) {
       if (row_valid) {
         m_in_nat = p.m_state[srow];
@@ -449,7 +463,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         l = p.l_state[srow];
       }
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 32 && warp_active; ++c) {
         uint32_t u[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -465,7 +479,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
     uint32_t n = 0;
     bool ok = true;
-    while (cur.valid()) {
+    while (warp_active && cur.valid()) {
       if (tile_visible(q, cur.k0, p.causal)) {
         if (!mbar_wait(BAR_S(t), n & 1u, abort_flag)) {
           ok = false;
@@ -486,7 +500,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         if (tile_needs_mask(q, cur.k0, cur.kend, p.causal)) {
           const int kvis = cur.kend - cur.k0;  // keys inside the chunk / range
           // Last key (tile-relative) this row sees under causal masking.
-          const long long kc = p.causal ? (long long)q.kmin + rloc - cur.k0 : (long long)kTileN;
+          const long long kc = p.causal ? (long long)q.kmin + tl - cur.k0 : (long long)kTileN;
           const int kcausal = (int)(kc < -1 ? -1 : (kc > kTileN ? kTileN : kc));
           const int klast = min(kvis - 1, kcausal);
 #pragma unroll
@@ -568,11 +582,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 
     // ------------------------------ epilogue ------------------------------
     if (ok && n > 0) ok = mbar_wait(BAR_O(t), 0, abort_flag);
-    if (ok) {
+    if (ok && warp_active) {
       tc_fence_after();
       if (MODE == kModeFinal || MODE == kModeSplit) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        const long long ooff = (((long long)(MODE == kModeSplit ? sigma * p.B + b : b) * p.N_q + row) * p.Hq + h) * D;
+        const long long ooff =
+            (((long long)(MODE == kModeSplit ? sigma * p.B + b : b) * p.N_q + row) * p.Hq + head) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float r[32];
@@ -605,9 +620,9 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         if (row_valid) {
           const float lse_v = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
           if (MODE == kModeSplit)
-            p.lse_part[(((long long)sigma * p.B + b) * p.Hq + h) * p.N_q + row] = lse_v;
+            p.lse_part[(((long long)sigma * p.B + b) * p.Hq + head) * p.N_q + row] = lse_v;
           else
-            p.lse[((long long)b * p.Hq + h) * p.N_q + row] = lse_v;
+            p.lse[((long long)b * p.Hq + head) * p.N_q + row] = lse_v;
         }
       } else if (n > 0) {  // kModeState with at least one visible tile
         // Hand back the state relative to the true running max.
@@ -669,12 +684,12 @@ cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) 
   return count_launch(cudaGetLastError());
 }
 
-CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N, int B) {
+CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N, int B, int box_heads = 1) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return CUDA_ERROR_NOT_FOUND;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)(128 / box_heads), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -683,11 +698,29 @@ CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N,
 
 }  // namespace
 
+Sm100Geometry sm100_geometry(const ProblemArgs& a, int mode) {
+  Sm100Geometry g;
+  const int G = a.Hq / a.Hkv;
+  // Pack the G query heads of a KV head into one tile when all of a KV
+  // head's query rows fit: one CTA then streams that KV once for the group.
+  const bool pack = mode != kModeState && G > 1 && (128 % G) == 0 && a.N_q * G <= kTileM;
+  g.gpack = pack ? G : 1;
+  g.gshift = 0;
+  while ((1 << g.gshift) < g.gpack) ++g.gshift;
+  g.tpt = kTileM / g.gpack;
+  g.two = a.N_q * g.gpack > kTileM;  // two query tiles per CTA share each K/V tile
+  const long long tok_per_cta = (long long)(g.two ? 2 : 1) * g.tpt;
+  g.n_qblk = (int)((a.N_q + tok_per_cta - 1) / tok_per_cta);
+  g.ctas_per_split = (long long)g.n_qblk * a.B * a.Hkv * (pack ? 1 : G);
+  return g;
+}
+
 cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   if (a.B <= 0 || a.N_q <= 0) return cudaSuccess;
+  const Sm100Geometry geo = sm100_geometry(a, mode);
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
-  if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B) != CUDA_SUCCESS ||
+  if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B, geo.gpack) != CUDA_SUCCESS ||
       encode_map(&prm.tm_k, a.k, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS ||
       encode_map(&prm.tm_v, a.v, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -713,11 +746,12 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   prm.S = mode == kModeSplit ? a.S : 1;
   prm.steps_per_split = (a.P + prm.S - 1) / prm.S;
   prm.out_f32 = a.out_f32;
-
-  const bool two = a.N_q > kTileM;  // two query tiles per CTA share each K/V tile
-  const int rows_per_cta = two ? 2 * kTileM : kTileM;
-  prm.n_qblk = (int)((a.N_q + rows_per_cta - 1) / rows_per_cta);
-  const long long grid = (long long)prm.n_qblk * a.B * a.Hq * prm.S;
+  prm.gpack = geo.gpack;
+  prm.gshift = geo.gshift;
+  prm.tpt = geo.tpt;
+  prm.n_qblk = geo.n_qblk;
+  const bool two = geo.two;
+  const long long grid = geo.ctas_per_split * prm.S;
   // K/V ring depth: as many 128-key slots as shared memory allows
   // (d=128: 2 query tiles + 5 slots = 224 KB; 1 tile + 6 slots).
 #define RA_LAUNCH(D_, NQT_, NS_)                                                  \

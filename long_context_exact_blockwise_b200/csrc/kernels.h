@@ -55,6 +55,17 @@ struct ProblemArgs {
 // Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.
 cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
 
+// CTA geometry the tensor-core path uses for a problem: query heads packed
+// per tile (gpack), tokens per tile, one or two query tiles per CTA, and the
+// number of CTAs per KV split.
+struct Sm100Geometry {
+  int gpack, gshift, tpt;
+  bool two;
+  int n_qblk;
+  long long ctas_per_split;
+};
+Sm100Geometry sm100_geometry(const ProblemArgs& a, int mode);
+
 // CUDA-core float32 path (also serves float32 block steps).
 cudaError_t launch_fwd_simt_f32(const ProblemArgs& a, int mode, cudaStream_t stream);
 

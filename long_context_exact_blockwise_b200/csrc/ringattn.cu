@@ -201,8 +201,7 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
 
   // Incremental query: split the ring steps over S CTAs per query block and
   // merge the partials by their log-sum-exp weights.
-  const long long rows_per_cta = N_q > 128 ? 256 : 128;
-  const long long items = (long long)B * Hq * ((N_q + rows_per_cta - 1) / rows_per_cta);
+  const long long items = sm100_geometry(a, kModeSplit).ctas_per_split;
   const int S = choose_splits(items, P, num_sms, N_q);
   if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd");
 
@@ -379,8 +378,7 @@ extern "C" int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v
   a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.S = 1; a.out_f32 = 0;
 
   // Same split count as ring_attn_fwd, so both produce the same partials.
-  const long long rows_per_cta = N_q > 128 ? 256 : 128;
-  const long long items = (long long)B * Hq * ((N_q + rows_per_cta - 1) / rows_per_cta);
+  const long long items = sm100_geometry(a, kModeSplit).ctas_per_split;
   const int S = choose_splits(items, P, num_sms, N_q);
   if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd_noalloc");
 

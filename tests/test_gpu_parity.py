@@ -37,6 +37,26 @@ def test_prefill_bf16(B, Hq, Hkv, N, d, causal, P):
     check_workload(w)
 
 
+PACKED_CASES = [
+    # Query heads of a KV group packed into one tile (G * N_q <= 128).
+    # (B, Hq, Hkv, N_q, N_kv, cache_idx, d, P, causal)
+    (1, 8, 1, 16, 16, -1, 128, 2, True),       # packed prefill, G = 8
+    (1, 4, 1, 30, 30, -1, 64, 3, True),        # packed prefill, G = 4, chunk 10
+    (2, 16, 2, 3, 1024, 1021, 128, 8, True),   # decode, G = 8
+    (1, 16, 1, 8, 2048, 2040, 128, 16, True),  # decode, G = 16, 128 rows
+    (1, 4, 2, 33, 512, 400, 128, 4, True),     # G = 2, 66 rows, unaligned cache_idx
+    (1, 8, 2, 7, 768, 300, 64, 6, False),      # non-causal incremental, G = 4
+]
+
+
+@pytest.mark.parametrize("splits", ["", "1", "5"])
+@pytest.mark.parametrize("B,Hq,Hkv,N_q,N_kv,ci,d,P,causal", PACKED_CASES)
+def test_packed_heads_bf16(monkeypatch, splits, B, Hq, Hkv, N_q, N_kv, ci, d, P, causal):
+    monkeypatch.setenv("RINGATTN_SPLITS", splits)
+    w = W(B=B, Hq=Hq, Hkv=Hkv, N_q=N_q, N_kv=N_kv, cache_idx=ci, d=d, causal=causal, P=P, seed=3 * N_q + Hq)
+    check_workload(w)
+
+
 def test_prefill_bf16_peaky_keys():
     # Keys scaled by 4 (exact) give logits with std ~4: a sharply peaked softmax.
     check_workload(W(Hq=4, Hkv=2, N_q=512, d=128, causal=True, P=4, k_scale=4.0, seed=11))
