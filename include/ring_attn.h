@@ -179,6 +179,17 @@ int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out
  */
 int ring_attn_sync_status(void* stream);
 
+/*
+ * ring_attn_exp2_poly -- y[i] = 2^x[i] evaluated the way the bf16 forward
+ * evaluates part of its softmax exponentials on FMA units instead of the
+ * special-function unit: x = n + f (n = round(x)), 2^f by a degree-3
+ * minimax polynomial on [-1/2, 1/2] (max relative error 7.5e-5), 2^n by an
+ * exponent-field add; inputs below -125 are clamped to -125.  Valid for
+ * x <= 127.  Exposed so the polynomial can be checked against the
+ * hardware exp2.  x, y: n floats of device memory.
+ */
+int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 /* Static description of a status code. Never NULL. */
 const char* ring_attn_error_string(int status);
 

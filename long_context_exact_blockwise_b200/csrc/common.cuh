@@ -248,6 +248,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 2^x on the FMA pipe for a pair of floats, for x <= 2^21 (inputs below -125
+// are clamped to -125, i.e. return about 2^-125 instead of a smaller value).
+// Range reduction x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n
+// in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a degree-3 minimax
+// polynomial (max relative error 7.5e-5, fitted by fit_exp2_poly.py); 2^n by
+// adding n to the exponent field.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(0.05517222f, 0.05517222f), f, make_float2(0.24261115f, 0.24261115f));
+  p = __ffma2_rn(p, f, make_float2(0.69326085f, 0.69326085f));
+  p = __ffma2_rn(p, f, make_float2(0.99992806f, 0.99992806f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

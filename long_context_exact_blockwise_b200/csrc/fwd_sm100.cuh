@@ -17,7 +17,9 @@
 //   warp 1       MMA issuer (one thread): S_t = Q_t K_j^T into TMEM
 //                (tcgen05.mma, A and B from smem), then O_t += P_t V_j with
 //                P_t read from TMEM.  Q tiles ping-pong: S for one tile is
-//                computed while the other tile's softmax runs.
+//                computed while the other tile's softmax runs.  (One issuer
+//                for both tiles measured faster than one per tile: MMAs of
+//                two threads interleave in the tensor pipe.)
 //   warp 2       TMEM allocator.
 //   warps 4..    one softmax warpgroup per query tile: thread = query row
 //                (TMEM lane).  Reads S with tcgen05.ld, masks (only tiles
@@ -35,6 +37,7 @@
 
 #pragma once
 
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -48,6 +51,13 @@ constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
 // The exponent base may trail the running row max by up to this much (log2
 // units) before O is rescaled: P entries stay <= 2^8, far inside bf16 range.
 constexpr float kRescaleSlack = 8.f;
+// Which of every 8 exponential pairs of an unmasked tile go to the FMA pipe
+// (bit i: pairs with index i mod 8).
+#ifndef RA_EXP2_POLY_MASK
+#define RA_EXP2_POLY_MASK 0x00
+#endif
+constexpr int kExp2PolyMask = RA_EXP2_POLY_MASK;
+
 // Register split of the two-query-tile kernel (384 threads at 168 registers).
 constexpr int kLaunchRegs = 168;
 constexpr int kRegsControl = 88;   // warps 0-3: TMA, MMA issue, TMEM allocation
@@ -151,8 +161,9 @@ struct Layout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kQOff + NQT * kTileBytes;
   static constexpr int kBarOff = kKVOff + NSLOT * kTileBytes;
-  // barriers: q, kv_full[NSLOT], kv_empty[NSLOT], s[NQT], p[NQT], o[NQT], drain
-  static constexpr int kNumBars = 1 + 2 * NSLOT + 3 * NQT + 1;
+  // barriers: q, kv_full[NSLOT], kv_empty[NSLOT], s[NQT], s_consumed[NQT],
+  // p_lo[NQT], p_hi[NQT], o[NQT], drain
+  static constexpr int kNumBars = 1 + 2 * NSLOT + 5 * NQT + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr uint32_t kTmemCols = (NQT * (128 + D) <= 256) ? 256 : 512;
@@ -183,12 +194,92 @@ __device__ __forceinline__ bool tile_needs_mask(const QTile& q, int k0, int kend
   return (kend - k0 < kTileN) || (causal && kend - 1 > q.kmin);
 }
 
+// P = exp2(sl * s - base) for keys [64 H, 64 H + 64) of one row, written as
+// bf16 pairs to TMEM columns [32 H, 32 H + 32) of S; returns the sum of the
+// float values.  Bit i of EMU set: pairs whose index is i mod 8 use
+// exp2_poly2 (FMA pipe) instead of ex2 (MUFU).  EMU is a compile-time
+// constant so each pair's choice is fixed in the generated code.
+template <int EMU, int H>
+__device__ __forceinline__ float softmax_p_half(const float (&s)[128], float sl, float base, uint32_t s_tmem) {
+  const float2 sl2 = make_float2(sl, sl);
+  const float2 nb2 = make_float2(-base, -base);
+  float2 sum0 = make_float2(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
+#pragma unroll
+  for (int c = 2 * H; c < 2 * H + 2; ++c) {
+    uint32_t u[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+      float2 e[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        e[k] = __ffma2_rn(make_float2(s[c * 32 + 2 * (i + k)], s[c * 32 + 2 * (i + k) + 1]), sl2, nb2);
+        if ((EMU >> ((i + k) & 7)) & 1)
+          e[k] = exp2_poly2(e[k]);
+        else
+          e[k] = make_float2(ex2(e[k].x), ex2(e[k].y));
+        u[i + k] = pack_bf16x2(e[k].x, e[k].y);
+      }
+      sum0 = __fadd2_rn(sum0, e[0]);
+      sum1 = __fadd2_rn(sum1, e[1]);
+      sum2 = __fadd2_rn(sum2, e[2]);
+      sum3 = __fadd2_rn(sum3, e[3]);
+    }
+    tmem_st16(s_tmem + c * 16, u);
+  }
+  const float2 sa = __fadd2_rn(__fadd2_rn(sum0, sum1), __fadd2_rn(sum2, sum3));
+  return sa.x + sa.y;
+}
+
+// S (+)= Q K^T for keys [64 H0, 64 H1) of a 128-key K tile at smem address
+// `kaddr`, into TMEM columns [64 H0, 64 H1) of the S tile at `s_tmem`.
+// Q and K are K-major with 128-byte swizzle: a K-step of 16 elements is 32
+// bytes inside a swizzle row, every 64 elements move to the next
+// 128-row x 128-byte block, and key row r starts r * 128 bytes into a block.
+template <int D, int H0, int H1>
+__device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint64_t qdesc, uint32_t kaddr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kTileM, (H1 - H0) * 64, 0);
+  const uint64_t kdesc = smem_desc_sw128(kaddr + H0 * 64 * 128, 16, 1024);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * (kTileM * 128) + (kk % 4) * 32;
+    umma_ss(s_tmem + 64 * H0, qdesc + (off >> 4), kdesc + (off >> 4), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V for keys [64 HALF, 64 HALF + 64) of a 128-key V tile at `vaddr`.
+// P (bf16 pairs) is read from TMEM at `p_tmem`: 16 keys = 8 columns.  For
+// B = V (N = d, K = keys) the tile is MN-major: 64-element blocks of d are
+// kTileN * 128 bytes apart (LBO), groups of 8 keys 1024 bytes apart (SBO),
+// 16 keys = 2048 bytes.
+template <int D, int HALF>
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t vaddr, bool accumulate_first) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kTileM, D, 1);
+  const uint64_t vdesc = smem_desc_sw128(vaddr, kTileN * 128, 1024);
+#pragma unroll
+  for (int kk = 4 * HALF; kk < 4 * HALF + 4; ++kk)
+    umma_ts(o_tmem, p_tmem + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (accumulate_first || kk > 0) ? 1u : 0u);
+}
+
+// Signal a per-warp barrier after this thread's tcgen05 operations: every
+// thread waits for and fences its own, the warp synchronises, one lane arrives.
+__device__ __forceinline__ void warp_arrive_after_tc(uint32_t bar, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 template <int D, int NQT, int NSLOT, int MODE>
 __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using L = Layout<D, NQT, NSLOT>;
   constexpr int kHalves = D / 64;  // 64-element (128-byte) swizzle columns per tile
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(kTileM, kTileN, 0);
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, 1);
+  // Single-tile CTAs (short or packed queries) have no second tile to keep
+  // the tensor pipe busy during a softmax, so they overlap inside the tile:
+  // the next S is computed in two halves (keys 64..127 while the softmax
+  // runs) and P is published in two halves (PV on keys 0..63 overlaps the
+  // rest of the softmax).  Two-tile CTAs ping-pong instead; the extra
+  // signalling measured slower there.
+  constexpr bool kSplitS = (NQT == 1);
+  constexpr bool kSplitPV = (NQT == 1);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -197,10 +288,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   auto BAR_Q = [&]() { return bar0; };
   auto BAR_KV_FULL = [&](int i) { return bar0 + 8u * (1 + i); };
   auto BAR_KV_EMPTY = [&](int i) { return bar0 + 8u * (1 + NSLOT + i); };
-  auto BAR_S = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + t); };
-  auto BAR_P = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + NQT + t); };
-  auto BAR_O = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 2 * NQT + t); };
-  const uint32_t BAR_DRAIN = bar0 + 8u * (1 + 2 * NSLOT + 3 * NQT);
+  auto BAR_S = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + t); };             // S_t in TMEM
+  auto BAR_SC = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + NQT + t); };      // S_t read by softmax
+  auto BAR_PA = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 2 * NQT + t); };  // P_t keys 0..63
+  auto BAR_PB = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 3 * NQT + t); };  // P_t keys 64..127, O ready
+  auto BAR_O = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 4 * NQT + t); };
+  const uint32_t BAR_DRAIN = bar0 + 8u * (1 + 2 * NSLOT + 5 * NQT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -224,8 +317,8 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   const int h = hk * p.G + g;
 
   QTile qt[NQT];
-#pragma unroll
   const long long qk_delta = p.q_pos0 - p.k_pos0;
+#pragma unroll
   for (int t = 0; t < NQT; ++t) qt[t] = make_qtile<NQT>(qblk, t, p.N_q, qk_delta, p.tpt, p.gshift);
   // Keys past the block's last query position are invisible to every row.
   int kmax_last = qt[0].kmax;
@@ -247,10 +340,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
       mbar_init(BAR_KV_EMPTY(i), 1);
     }
     for (int t = 0; t < NQT; ++t) {
-      // One arrival per thread of the softmax warps that hold valid rows.
+      // One arrival per softmax warp that holds valid rows.
       const int active_warps = min(4, (qt[t].nv + 31) / 32);
       mbar_init(BAR_S(t), 1);
-      mbar_init(BAR_P(t), 32 * max(1, active_warps));
+      mbar_init(BAR_SC(t), max(1, active_warps));
+      mbar_init(BAR_PA(t), max(1, active_warps));
+      mbar_init(BAR_PB(t), max(1, active_warps));
       mbar_init(BAR_O(t), 1);
     }
     mbar_init(BAR_DRAIN, 1);
@@ -334,39 +429,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
         qdesc[t] = smem_desc_sw128(sbase + L::kQOff + t * L::kTileBytes, 16, 1024);
-      auto issue_s = [&](int t, uint32_t kslot) {
-        const uint32_t kaddr = sbase + L::kKVOff + kslot * L::kTileBytes;
-        const uint64_t kdesc = smem_desc_sw128(kaddr, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // K-step of 16 elements = 32 bytes inside a 128-byte swizzle row;
-          // every 64 elements move to the next 128-row x 128-byte block.
-          const uint32_t off = (kk / 4) * (kTileM * 128) + (kk % 4) * 32;
-          umma_ss(tmem + 128 * t, qdesc[t] + (off >> 4), kdesc + (off >> 4), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(BAR_S(t));
-      };
-      auto issue_pv = [&](int t, uint32_t vslot, bool accumulate_first) {
-        const uint32_t vaddr = sbase + L::kKVOff + vslot * L::kTileBytes;
-        // V tile: keys are rows (128 bytes of d per row and 64-element
-        // column block); for B = V (N = d, K = keys) that is MN-major:
-        // 64-element blocks of d are kTileN*128 bytes apart (LBO), groups of
-        // 8 keys are 1024 bytes apart (SBO).
-        const uint64_t vdesc = smem_desc_sw128(vaddr, kTileN * 128, 1024);
-        const uint32_t o_tmem = tmem + 128 * NQT + D * t;
-        const uint32_t p_tmem = tmem + 128 * t;
-#pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk) {
-          // 16 keys per MMA: 2048 bytes of V; 8 TMEM columns of packed P.
-          umma_ts(o_tmem, p_tmem + kk * 8, vdesc + ((kk * 2048) >> 4), kIdescPV,
-                  (accumulate_first || kk > 0) ? 1u : 0u);
-        }
-      };
-      uint32_t p_seen[NQT];
+      auto kv_addr = [&](uint32_t slot) { return sbase + L::kKVOff + slot * L::kTileBytes; };
+      uint32_t n_seen[NQT];  // visible tiles of query tile t handled so far
       bool o_live[NQT];
 #pragma unroll
       for (int t = 0; t < NQT; ++t) {
-        p_seen[t] = 0;
+        n_seen[t] = 0;
         o_live[t] = (MODE == kModeState);
       }
       KvCursor cur;
@@ -378,46 +446,83 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         if (ok) {
 #pragma unroll
           for (int t = 0; t < NQT; ++t)
-            if (tile_visible(qt[t], cur.k0, p.causal)) issue_s(t, 0);
+            if (tile_visible(qt[t], cur.k0, p.causal)) {
+              mma_qk<D, 0, 2>(tmem + 128 * t, qdesc[t], kv_addr(0));
+              tc_commit(BAR_S(t));
+            }
           tc_commit(BAR_KV_EMPTY(0));
         }
       }
+      // Per query tile t and KV tile j (both visible), in issue order:
+      //   [softmax read S(j)]  S(j+1) keys 64..127 -> S columns 64..127
+      //                        (single-tile CTAs only: with two tiles the
+      //                        other tile's work fills the tensor pipe)
+      //   [P keys 0..63]       PV(j) keys 0..63
+      //   [P keys 64..127]     PV(j) keys 64..127, then S(j+1) (keys 0..63
+      //                        only if the other half went early) into the
+      //                        S columns, after PV has read P.
+
       while (ok && cur.valid()) {
         KvCursor nxt = cur;
         nxt.next();
         const bool has_next = nxt.valid();
         const uint32_t vfill = 2 * j + 1, kfill = 2 * j + 2;
-        ok = mbar_wait(BAR_KV_FULL(vfill % NSLOT), (vfill / NSLOT) & 1u, abort_flag);
+        const uint32_t vslot = vfill % NSLOT, kslot = kfill % NSLOT;
+        ok = mbar_wait(BAR_KV_FULL(vslot), (vfill / NSLOT) & 1u, abort_flag);
         tc_fence_after();
         bool k_ready = false;
+        auto wait_k = [&]() {
+          if (!k_ready) {
+            ok = mbar_wait(BAR_KV_FULL(kslot), (kfill / NSLOT) & 1u, abort_flag);
+            tc_fence_after();
+            k_ready = true;
+          }
+          return ok;
+        };
 #pragma unroll
         for (int t = 0; t < NQT && ok; ++t) {
-          if (tile_visible(qt[t], cur.k0, p.causal)) {
-            ok = mbar_wait(BAR_P(t), p_seen[t] & 1u, abort_flag);
-            ++p_seen[t];
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, vfill % NSLOT, o_live[t]);
-            o_live[t] = true;
-          }
-          if (has_next && tile_visible(qt[t], nxt.k0, p.causal)) {
-            if (!k_ready) {
-              ok = mbar_wait(BAR_KV_FULL(kfill % NSLOT), (kfill / NSLOT) & 1u, abort_flag);
-              if (!ok) break;
+          const bool vc = tile_visible(qt[t], cur.k0, p.causal);
+          const bool vn = has_next && tile_visible(qt[t], nxt.k0, p.causal);
+          if (vc) {
+            const uint32_t par = n_seen[t] & 1u;
+            ++n_seen[t];
+            if (kSplitS && vn) {
+              if (!wait_k()) break;
+              if (!(ok = mbar_wait(BAR_SC(t), par, abort_flag))) break;
               tc_fence_after();
-              k_ready = true;
+              mma_qk<D, 1, 2>(tmem + 128 * t, qdesc[t], kv_addr(kslot));
             }
-            issue_s(t, kfill % NSLOT);
+            if (kSplitPV) {
+              if (!(ok = mbar_wait(BAR_PA(t), par, abort_flag))) break;
+              tc_fence_after();
+              mma_pv<D, 0>(tmem + 128 * NQT + D * t, tmem + 128 * t, kv_addr(vslot), o_live[t]);
+            }
+            if (!(ok = mbar_wait(BAR_PB(t), par, abort_flag))) break;
+            tc_fence_after();
+            if (!kSplitPV) mma_pv<D, 0>(tmem + 128 * NQT + D * t, tmem + 128 * t, kv_addr(vslot), o_live[t]);
+            mma_pv<D, 1>(tmem + 128 * NQT + D * t, tmem + 128 * t, kv_addr(vslot), true);
+            o_live[t] = true;
+            if (vn) {
+              if (kSplitS) {
+                mma_qk<D, 0, 1>(tmem + 128 * t, qdesc[t], kv_addr(kslot));
+              } else {
+                if (!wait_k()) break;
+                mma_qk<D, 0, 2>(tmem + 128 * t, qdesc[t], kv_addr(kslot));
+              }
+              tc_commit(BAR_S(t));
+            }
+          } else if (vn) {
+            // S_t is free: its last P was consumed by a PV issued earlier.
+            if (!wait_k()) break;
+            mma_qk<D, 0, 2>(tmem + 128 * t, qdesc[t], kv_addr(kslot));
+            tc_commit(BAR_S(t));
           }
         }
         if (!ok) break;
-        tc_commit(BAR_KV_EMPTY(vfill % NSLOT));
+        tc_commit(BAR_KV_EMPTY(vslot));
         if (has_next) {
-          if (!k_ready) {  // every tile the cursor yields is visible to some query tile
-            ok = mbar_wait(BAR_KV_FULL(kfill % NSLOT), (kfill / NSLOT) & 1u, abort_flag);
-            tc_fence_after();
-          }
-          tc_commit(BAR_KV_EMPTY(kfill % NSLOT));
+          if (!wait_k()) break;  // every tile the cursor yields is visible to some query tile
+          tc_commit(BAR_KV_EMPTY(kslot));
         }
         cur = nxt;
         ++j;
@@ -493,11 +598,15 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
           tmem_ld32(s_tmem + c * 32, r);
         }
         tc_wait_ld();
+        // S is in registers: the issuer may now overwrite its columns 64..127
+        // with the next tile's scores (the first 64 columns get P).
+        if constexpr (kSplitS) warp_arrive_after_tc(BAR_SC(t), lane);
         if (!fold) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] *= p.scale_log2;
         }
-        if (tile_needs_mask(q, cur.k0, cur.kend, p.causal)) {
+        const bool masked = tile_needs_mask(q, cur.k0, cur.kend, p.causal);
+        if (masked) {
           const int kvis = cur.kend - cur.k0;  // keys inside the chunk / range
           // Last key (tile-relative) this row sees under causal masking.
           const long long kc = p.causal ? (long long)q.kmin + tl - cur.k0 : (long long)kTileN;
@@ -524,57 +633,37 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
           l *= alpha;
         }
         const float base = (m2 == -INFINITY) ? 0.f : m2;
-        const float2 sl2 = make_float2(sl, sl);
-        const float2 nb2 = make_float2(-base, -base);
-        float2 sum0 = make_float2(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
-        // P = exp2(sl * s - base) as bf16 pairs over the first 64 columns of S.
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[16];
-#pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            float2 e0 = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), sl2, nb2);
-            float2 e1 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 2], s[c * 32 + 2 * i + 3]), sl2, nb2);
-            float2 e2 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 4], s[c * 32 + 2 * i + 5]), sl2, nb2);
-            float2 e3 = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 6], s[c * 32 + 2 * i + 7]), sl2, nb2);
-            e0 = make_float2(ex2(e0.x), ex2(e0.y));
-            e1 = make_float2(ex2(e1.x), ex2(e1.y));
-            e2 = make_float2(ex2(e2.x), ex2(e2.y));
-            e3 = make_float2(ex2(e3.x), ex2(e3.y));
-            sum0 = __fadd2_rn(sum0, e0);
-            sum1 = __fadd2_rn(sum1, e1);
-            sum2 = __fadd2_rn(sum2, e2);
-            sum3 = __fadd2_rn(sum3, e3);
-            u[i] = pack_bf16x2(e0.x, e0.y);
-            u[i + 1] = pack_bf16x2(e1.x, e1.y);
-            u[i + 2] = pack_bf16x2(e2.x, e2.y);
-            u[i + 3] = pack_bf16x2(e3.x, e3.y);
-          }
-          tmem_st16(s_tmem + c * 16, u);
-        }
-        const float2 sa = __fadd2_rn(__fadd2_rn(sum0, sum1), __fadd2_rn(sum2, sum3));
-        l += sa.x + sa.y;
+        // O must be rescaled before the first half of P is published: the
+        // PV for keys 0..63 accumulates into it.
         const bool o_has_data = (MODE == kModeState) || n > 0;
         if (o_has_data && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; c += 2) {
-            float r0[32], r1[32];
-            tmem_ld32(o_tmem + c * 32, r0);
-            tmem_ld32(o_tmem + (c + 1) * 32, r1);
+          // Rare (the max must jump past the slack): one 32-column chunk at
+          // a time, in place, while the scores still occupy registers.
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float r[32];
+            tmem_ld32(o_tmem + c * 32, r);
             tc_wait_ld();
-            uint32_t u0[32], u1[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              u0[i] = __float_as_uint(r0[i] * alpha);
-              u1[i] = __float_as_uint(r1[i] * alpha);
-            }
-            tmem_st32(o_tmem + c * 32, u0);
-            tmem_st32(o_tmem + (c + 1) * 32, u1);
+            for (int i = 0; i < 32; ++i) r[i] *= alpha;
+            tmem_st32(o_tmem + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(r));
           }
         }
+        // P in two halves (published separately for single-tile CTAs).
+        // Unmasked tiles may evaluate part of their
+        // exponentials on the FMA pipe; masked tiles use ex2 throughout so
+        // masked keys contribute exactly zero.
+        float rs = masked ? softmax_p_half<0, 0>(s, sl, base, s_tmem)
+                          : softmax_p_half<kExp2PolyMask, 0>(s, sl, base, s_tmem);
+        if constexpr (kSplitPV) {
+          tc_wait_st();
+          warp_arrive_after_tc(BAR_PA(t), lane);
+        }
+        rs += masked ? softmax_p_half<0, 1>(s, sl, base, s_tmem)
+                     : softmax_p_half<kExp2PolyMask, 1>(s, sl, base, s_tmem);
         tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(BAR_P(t));
+        warp_arrive_after_tc(BAR_PB(t), lane);
+        l += rs;
         ++n;
       }
       cur.next();

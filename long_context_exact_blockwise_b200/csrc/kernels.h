@@ -77,6 +77,9 @@ cudaError_t launch_finalize(const float* acc, const float* m, const float* l, vo
 cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse,
                              int B, int Hq, long long N_q, int d, int out_f32, cudaStream_t stream);
 
+// y = exp2_poly2(x) elementwise (the FMA-pipe exp2 of the softmax), for tests.
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
+
 // Resolve cuTensorMapEncodeTiled through the runtime (no link-time libcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,

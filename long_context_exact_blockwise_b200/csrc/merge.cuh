@@ -133,7 +133,25 @@ finalize_kernel(const float* __restrict__ acc, const float* __restrict__ m, cons
   if (lane == 0) lse[r] = lr > 0.f ? mr + logf(lr) : -INFINITY;
 }
 
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const long long pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(x, y, n);
+  return count_launch(cudaGetLastError());
+}
 
 cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse, int B,
                              int Hq, long long N_q, int d, int out_f32, cudaStream_t st) {

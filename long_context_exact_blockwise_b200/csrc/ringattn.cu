@@ -309,6 +309,15 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
                 "lse_merge");
 }
 
+int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0) return RA_ERR_INVALID_ARG;
+  if (n == 0) return RA_OK;
+  int r = check_device(nullptr);
+  if (r != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return finish(launch_exp2_poly(x, y, n, st), st, "ring_attn_exp2_poly");
+}
+
 }  // extern "C"
 
 // ----------------------------------------------------------------------------

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
     "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_block_step", "ring_attn_finalize",
-    "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count",
+    "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
     "RA_ERR_OOM", "RA_DTYPE_BF16", "RA_DTYPE_F32",
@@ -62,6 +62,7 @@ _SIGS = {
     "ring_attn_last_error": [],
     "ring_attn_version": [],
     "ring_attn_launch_count": [],
+    "ring_attn_exp2_poly": [_p, _p, _l, _p],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -108,6 +109,14 @@ def ring_attn_error_string(status: int) -> str:
 
 def ring_attn_version() -> int:
     return lib.ring_attn_version()
+
+
+def ring_attn_exp2_poly(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """2^x by the softmax's FMA-pipe polynomial (for checking its error)."""
+    _need(x, "x", torch.float32)
+    y = torch.empty_like(x) if out is None else out
+    _check(lib.ring_attn_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream, x.device)), "ring_attn_exp2_poly")
+    return y
 
 
 def ring_attn_launch_count() -> int:

@@ -250,3 +250,30 @@ def test_invalid_call_launches_nothing():
     with pytest.raises(R.RingAttnError) as ei:
         R.ring_attn_fwd(q, q, q, causal=True, P=3, chunk=33)
     assert ei.value.status == R.RA_ERR_INVALID_ARG
+
+
+def test_exp2_poly_error_bound():
+    # The FMA-pipe exp2 of the softmax against the hardware exp2 (torch.exp2
+    # on CUDA): relative error within the fitted minimax bound 7.5e-5 plus
+    # float32 rounding, over the exponent range the softmax uses.
+    R = ra()
+    g = torch.Generator(device="cuda").manual_seed(0)
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001, device="cuda"),
+                   torch.rand(1_000_000, device="cuda", generator=g) * 30 - 25,
+                   torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, -124.5, 7.5], device="cuda")])
+    y = R.ring_attn_exp2_poly(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref) / ref).abs().max().item()
+    assert rel <= 7.6e-5, rel
+    # Below the clamp the result is 2^-125 up to the same relative error.
+    z = R.ring_attn_exp2_poly(torch.tensor([-200.0, -1e30], device="cuda"))
+    assert torch.allclose(z.double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64, device="cuda"),
+                          rtol=1e-4, atol=0)
+
+
+@pytest.mark.parametrize("mask", ["0x11", "0x55", "0xff"])
+def test_prefill_with_fma_exp2(monkeypatch, mask):
+    monkeypatch.setenv("RINGATTN_EMU_MASK", mask)
+    check_workload(W(B=1, Hq=4, Hkv=2, N_q=1024, d=128, causal=True, P=4, seed=61))
+    check_workload(W(B=1, Hq=2, Hkv=2, N_q=512, d=64, causal=False, P=2, k_scale=4.0, seed=62))
+    check_workload(W(B=2, Hq=8, Hkv=2, N_q=96, N_kv=2048, cache_idx=1952, d=128, causal=True, P=8, seed=63))

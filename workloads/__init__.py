@@ -73,6 +73,10 @@ CONFIGS = {
                     dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 1, seed=5100),
     "5d8": Workload("cache_idx_decode_Nq8_Nkv262144", B=4, Hq=32, Hkv=8, N_q=8, N_kv=262144, d=128,
                     dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5200),
+    # A quarter-length decode cache (1.07 GB of K/V, still 8x the L2) for
+    # profiler captures that must stay small.
+    "5d1s": Workload("cache_idx_decode_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
+                     dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5300),
 }
 
 
