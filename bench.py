@@ -42,8 +42,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 12.351685 GB read + 0.402486 GB written.
-    "llama7b_prefill_N32768": {"bytes": 12.754171e9, "src": "72706bf42e83b2b0"},
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.828749 GB read + 0.258709 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.087458e9, "src": "2e7ad4d545362cff"},
+    # profiles/fwd_sm100_decode_Nq1_Nkv65536.md: 1.073881 GB read + 0.007975 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.081856e9, "src": "2e7ad4d545362cff"},
+    # The full-length decode scales the quarter-length capture by its 4x KV
+    # length (traffic is K/V streaming, proportional to N_kv).
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.081856e9, "src": "2e7ad4d545362cff"},
 }
 
 
