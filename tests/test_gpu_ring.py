@@ -1,0 +1,42 @@
+"""The ring driver with its default CUDA compute (block step + finalize
+kernels) on one GPU: a one-rank group runs the whole sequence as a single
+ring step, which must match the float64 oracle."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import oracle
+import workloads
+from parity_util import TOL_LSE, TOL_OUT
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture
+def one_rank_group():
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    yield
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_driver_cuda_compute(one_rank_group, dtype, causal):
+    from long_context_exact_blockwise_b200.ring import ring_attention
+    w = workloads.small(B=2, Hq=4, Hkv=2, N_q=384, d=128, dtype=dtype, causal=causal, P=1, seed=90)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    out, lse = ring_attention(q, k, v, causal=causal, scale=w.scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
+    assert np.max(np.abs(out.float().cpu().numpy() - ro)) <= TOL_OUT[dtype]
+    assert np.max(np.abs(lse.cpu().numpy() - rl)) <= TOL_LSE
