@@ -94,6 +94,26 @@ def hbm_bytes_of(w: workloads.Workload) -> float:
     return es * (2 * w.B * w.N_q * w.Hq * w.d + 2 * w.B * w.N_kv * w.Hkv * w.d) + 4 * w.B * w.Hq * w.N_q
 
 
+# ----------------------------------------------------------------- ranks
+def rank_seed(w: workloads.Workload, rank: int) -> int:
+    """Each replica draws its own inputs."""
+    return w.seed + 7919 * rank
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The slowest rank's time (or any maximum) across the process group."""
+    if not torch.distributed.is_initialized() or torch.distributed.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of every replica over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons via NVML while running."""
@@ -158,7 +178,7 @@ def run_ours(args, w, rank, world, device):
 
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    q, k, v = workloads.make_qkv(w, device=device, seed=w.seed + 7919 * rank)
+    q, k, v = workloads.make_qkv(w, device=device, seed=rank_seed(w, rank))
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.N_q), device=device, dtype=torch.float32)
     ci = None if w.cache_idx < 0 else w.cache_idx
@@ -196,12 +216,8 @@ def run_ours(args, w, rank, world, device):
     clocks.stop()
     barrier()
     launches = R.ring_attn_launch_count() - launches0
-    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), device)
     per_launch = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
     status = R.ring_attn_sync_status(stream)
     if status != 0:
         raise RuntimeError(f"device status word {status} after the timed region")
@@ -235,11 +251,7 @@ def run_ours(args, w, rank, world, device):
     b.record(stream)
     torch.cuda.synchronize(device)
     barrier()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, device)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
     res = dict(ms_total=ms_total, per_launch_ms=per_launch, launches=launches, clocks=clocks.summary(),
@@ -353,7 +365,7 @@ def main():
     device = local_rank
     res = run_ours(args, w, rank, world, device)
     ms_step = res["ms_total"] / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(flops, world, ms_step)
     launch_ms = statistics.mean(res["per_launch_ms"])
     achieved = flops / (launch_ms * 1e-3) / 1e12
     # A kernel timed alone for a short step is compared with the burst bf16
@@ -381,7 +393,7 @@ def main():
         cpu = {"value": f_ / s_ / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{r_} random (row, head) query rows in runs of 16 of this workload, {s_:.1f} s of "
                          f"float64 oracle work on the host"}
-    e2e_val = flops * world / (res["e2e_ms"] * 1e-3) / 1e12
+    e2e_val = aggregate_tflops(flops, world, res["e2e_ms"])
     line = {
         "metric": "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
