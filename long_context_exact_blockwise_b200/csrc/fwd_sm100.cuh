@@ -89,6 +89,8 @@ struct Sm100Params {
   int out_f32;
   int gpack;   // query heads packed into one tile (1, or G for incremental queries)
   int gshift;  // log2(gpack)
+  int skip_loads;  // failure-detection test: the producer issues no copies, so the
+                   // consumers' bounded waits expire and the kernel unwinds
   int tpt;     // tokens per tile: 128 / gpack
 };
 
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   }
   if (warp == 0) {
     // =========================== TMA producer ===========================
-    if (lane == 0) {
+    if (lane == 0 && !p.skip_loads) {
       prefetch_tmap(&p.tm_q);
       prefetch_tmap(&p.tm_k);
       prefetch_tmap(&p.tm_v);
@@ -837,6 +839,11 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   prm.out_f32 = a.out_f32;
   prm.gpack = geo.gpack;
   prm.gshift = geo.gshift;
+  {
+    // Host-side fault injection for the failure-detection test (see ringattn.cu).
+    const char* f = std::getenv("RINGATTN_FAULT");
+    prm.skip_loads = (f && std::strcmp(f, "device_wait") == 0) ? 1 : 0;
+  }
   prm.tpt = geo.tpt;
   prm.n_qblk = geo.n_qblk;
   const bool two = geo.two;

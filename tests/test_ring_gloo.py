@@ -102,3 +102,38 @@ def test_ring_visit_order_matches_schedule_figure():
     assert ring_visit_order(0, 4) == [0, 1, 2, 3]
     assert ring_visit_order(1, 4) == [1, 2, 3, 0]
     assert ring_visit_order(3, 4) == [3, 0, 1, 2]
+
+
+def _dying_worker(rank, world, port, results):
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # This rank leaves before the ring exchange starts (between steps).
+        os._exit(0)
+    from long_context_exact_blockwise_b200.ring import ring_attention
+    bs, fin, init = _oracle_compute()
+    q = torch.randn(1, 8, 2, 4, dtype=torch.float64)
+    try:
+        ring_attention(q, q.clone(), q.clone(), causal=False, scale=0.5, block_step=bs, finalize=fin,
+                       init_state=init)
+        results[rank] = "finished"
+    except Exception as e:  # the dead peer surfaces as an error, not a hang
+        results[rank] = "error: " + type(e).__name__
+
+
+def test_ring_peer_loss_surfaces_as_error():
+    ctx = mp.get_context("spawn")
+    results = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode is not None for p in procs), "a rank hung"
+    assert results.get(0, "").startswith("error"), dict(results)
