@@ -51,6 +51,10 @@ constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
 // The exponent base may trail the running row max by up to this much (log2
 // units) before O is rescaled: P entries stay <= 2^8, far inside bf16 range.
 constexpr float kRescaleSlack = 8.f;
+// Row sum of one tile's P with every entry <= 2^kRescaleSlack is at most
+// 128 * 2^8; a sum at most 2^8 guarantees every entry is, so the one-pass
+// path checks the sum against 2^8.
+constexpr float kSlackSum = 256.f;
 // Which of every 8 exponential pairs of an unmasked tile go to the FMA pipe
 // (bit i: pairs with index i mod 8).
 #ifndef RA_EXP2_POLY_MASK
@@ -617,52 +621,90 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = (c <= klast) ? s[c] : -INFINITY;
         }
-        // Row max: four independent chains of 3-input max.
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // After a row's first tile the exponentials use the current base m2
+        // directly: every P <= 2^kRescaleSlack exactly when the row sum is,
+        // and only a larger sum (rare) makes the tile compute its max and,
+        // if the max did jump past the slack, redo P with a new base before
+        // P is published.  A row's first tile, and single-tile CTAs (which
+        // publish half of P early), take the max first.
+        auto row_max = [&]() {
+          // Four independent chains of 3-input max.
+          float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
-          mx0 = fmax3(mx0, s[c], s[c + 1]);
-          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
-        }
-        const float m_tile = fmax3(fmaxf(mx0, mx1), mx2, mx3) * sl;  // -inf stays -inf (sl > 0)
-        m_true = fmaxf(m_true, m_tile);
+          for (int c = 4; c < 128; c += 8) {
+            mx0 = fmax3(mx0, s[c], s[c + 1]);
+            mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+            mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+            mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+          }
+          return fmax3(fmaxf(mx0, mx1), mx2, mx3) * sl;  // -inf stays -inf (sl > 0)
+        };
+        auto compute_p = [&](float base) {
+          // P in two halves (published separately for single-tile CTAs).
+          // Unmasked tiles may evaluate part of their exponentials on the
+          // FMA pipe; masked tiles use ex2 so masked keys give exactly 0.
+          float r = masked ? softmax_p_half<0, 0>(s, sl, base, s_tmem)
+                           : softmax_p_half<kExp2PolyMask, 0>(s, sl, base, s_tmem);
+          if constexpr (kSplitPV) {
+            tc_wait_st();
+            warp_arrive_after_tc(BAR_PA(t), lane);
+          }
+          r += masked ? softmax_p_half<0, 1>(s, sl, base, s_tmem)
+                      : softmax_p_half<kExp2PolyMask, 1>(s, sl, base, s_tmem);
+          return r;
+        };
+        // After a row's first tile, P is computed directly with the current
+        // base m2.  Every entry of P is <= 2^kRescaleSlack whenever the row
+        // sum is, so only a larger sum (rare) makes the tile compute its max;
+        // if that max did pass m2 + slack, O and l are rescaled and P is
+        // redone with the new base before it is published.  A row's first
+        // tile, and single-tile CTAs (which publish half of P early), take
+        // the max first.
+        float rs = 0.f;
         float alpha = 1.f;
-        if (m_tile > m2 + kRescaleSlack) {
-          alpha = ex2(m2 - m_tile);  // 0 when m2 = -inf
-          m2 = m_tile;
-          l *= alpha;
-        }
-        const float base = (m2 == -INFINITY) ? 0.f : m2;
-        // O must be rescaled before the first half of P is published: the
-        // PV for keys 0..63 accumulates into it.
-        const bool o_has_data = (MODE == kModeState) || n > 0;
-        if (o_has_data && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // Rare (the max must jump past the slack): one 32-column chunk at
-          // a time, in place, while the scores still occupy registers.
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float r[32];
-            tmem_ld32(o_tmem + c * 32, r);
-            tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] *= alpha;
-            tmem_st32(o_tmem + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(r));
+        bool max_first = kSplitPV || n == 0 || __any_sync(0xffffffffu, m2 == -INFINITY);
+        bool redo = max_first;
+        if (!max_first) {
+          rs = compute_p(m2);
+          if (__any_sync(0xffffffffu, !(rs <= kSlackSum))) {
+            const float m_tile = row_max();
+            m_true = fmaxf(m_true, m_tile);
+            if (m_tile > m2 + kRescaleSlack) {
+              alpha = ex2(m2 - m_tile);
+              m2 = m_tile;
+              l *= alpha;
+            }
+            redo = __any_sync(0xffffffffu, alpha != 1.f);
+          } else if (MODE == kModeState) {
+            m_true = fmaxf(m_true, row_max());  // to hand the state back at the true max
+          }
+        } else {
+          const float m_tile = row_max();
+          m_true = fmaxf(m_true, m_tile);
+          if (m_tile > m2 + kRescaleSlack) {
+            alpha = ex2(m2 - m_tile);  // 0 when m2 = -inf
+            m2 = m_tile;
+            l *= alpha;
           }
         }
-        // P in two halves (published separately for single-tile CTAs).
-        // Unmasked tiles may evaluate part of their
-        // exponentials on the FMA pipe; masked tiles use ex2 throughout so
-        // masked keys contribute exactly zero.
-        float rs = masked ? softmax_p_half<0, 0>(s, sl, base, s_tmem)
-                          : softmax_p_half<kExp2PolyMask, 0>(s, sl, base, s_tmem);
-        if constexpr (kSplitPV) {
-          tc_wait_st();
-          warp_arrive_after_tc(BAR_PA(t), lane);
+        if (redo) {
+          // O must be rescaled before P is published: PV accumulates into it.
+          const bool o_has_data = (MODE == kModeState) || n > 0;
+          if (o_has_data && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // Rare (the max must jump past the slack): one 32-column chunk at
+            // a time, in place, while the scores still occupy registers.
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              float r[32];
+              tmem_ld32(o_tmem + c * 32, r);
+              tc_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] *= alpha;
+              tmem_st32(o_tmem + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(r));
+            }
+          }
+          rs = compute_p((m2 == -INFINITY) ? 0.f : m2);
         }
-        rs += masked ? softmax_p_half<0, 1>(s, sl, base, s_tmem)
-                     : softmax_p_half<kExp2PolyMask, 1>(s, sl, base, s_tmem);
         tc_wait_st();
         warp_arrive_after_tc(BAR_PB(t), lane);
         l += rs;
