@@ -27,6 +27,7 @@ Parity status: every public function here is pinned by tests under
 routine, brute force, closed forms, invariants, the pages' printed schedule).
 """
 from .attention import (
+    attention_bwd_ref,
     attention_ref,
     block_step_ref,
     finalize_ref,
@@ -38,6 +39,7 @@ from .attention import (
 )
 
 __all__ = [
+    "attention_bwd_ref",
     "attention_ref",
     "block_step_ref",
     "finalize_ref",

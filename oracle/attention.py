@@ -270,3 +270,53 @@ def lse_merge_ref(o_parts, lse_parts):
     out = np.where(np.transpose(has, (0, 2, 1))[..., None], out, 0.0)
     lse = np.where(has, base + np.log(safe), NEG_INF)
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (gradients of the exact attention), by definition.
+# ---------------------------------------------------------------------------
+
+def attention_bwd_ref(q, k, v, dout, *, causal: bool, scale: float, cache_idx: int = -1):
+    """Gradients of out = attention(q, k, v) for an upstream gradient dout.
+
+    The pages define only the forward; they use it for training ([BT]
+    production parameters: Ring Attention with FSDP for 7B-13B models; [CI]
+    blockwise configuration with a gradient-checkpoint policy), so the
+    backward is the mathematical gradient of the forward definition above.
+
+    Per (b, query head h, row t) with visible keys J(t), writing
+    s_j = scale * q_t . k_j, p_j = softmax_j(s), o_t = sum_j p_j v_j:
+        dv_j  += p_tj * dout_t                      (summed over t and the
+        dp_tj  = dout_t . v_j                         query heads of the group)
+        D_t    = dout_t . o_t   ( = sum_j p_tj dp_tj )
+        ds_tj  = p_tj (dp_tj - D_t)
+        dq_t   = scale * sum_j ds_tj k_j
+        dk_j  += scale * ds_tj q_t
+    The softmax is recomputed here from the definition (full score rows).
+    Returns (dq [B, N_q, Hq, d], dk [B, N_kv, Hkv, d], dv [B, N_kv, Hkv, d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N_q, Hq, d = q.shape
+    N_kv, Hkv = k.shape[1], k.shape[2]
+    pos = _query_positions(N_q, cache_idx)
+    vis = _visible(pos, np.arange(N_kv, dtype=np.int64), causal)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            s = scale * (q[b, :, h, :] @ k[b, :, hk, :].T)
+            s = np.where(vis, s, NEG_INF)
+            w, m, l = _softmax_rows(s)
+            has = l > 0
+            p = np.zeros_like(w)
+            p[has] = w[has] / l[has, None]
+            o = p @ v[b, :, hk, :]
+            dp = do[b, :, h, :] @ v[b, :, hk, :].T
+            D = np.sum(do[b, :, h, :] * o, axis=1)
+            ds = p * (dp - D[:, None])
+            dv[b, :, hk, :] += p.T @ do[b, :, h, :]
+            dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
+            dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
+    return dq, dk, dv

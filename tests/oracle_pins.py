@@ -316,5 +316,57 @@ def pin_schedule(O):
             assert (ci // qcs) * qcs == ci
 
 
+def pin_backward_autograd(O):
+    # Gradients against torch autograd through float64 SDPA (explicit mask,
+    # GQA by repeating KV heads so autograd sums the group's gradients).
+    cases = [(2, 13, 13, 4, 2, 8, True, 0.3, -1), (1, 9, 9, 2, 2, 4, False, 0.7, -1),
+             (1, 5, 20, 4, 1, 8, True, 0.25, 15)]
+    for i, (B, N_q, N_kv, Hq, Hkv, d, causal, scale, ci) in enumerate(cases):
+        q = _rand((B, N_q, Hq, d), 130 + i).requires_grad_(True)
+        k = _rand((B, N_kv, Hkv, d), 140 + i).requires_grad_(True)
+        v = _rand((B, N_kv, Hkv, d), 150 + i).requires_grad_(True)
+        do = _rand((B, N_q, Hq, d), 160 + i)
+        G = Hq // Hkv
+        qpos = torch.arange(N_q) + (0 if ci < 0 else ci)
+        kpos = torch.arange(N_kv)
+        mask = (kpos[None, :] <= qpos[:, None]) if causal else torch.ones(N_q, N_kv, dtype=torch.bool)
+        out = F.scaled_dot_product_attention(q.transpose(1, 2), k.repeat_interleave(G, dim=2).transpose(1, 2),
+                                             v.repeat_interleave(G, dim=2).transpose(1, 2), attn_mask=mask,
+                                             scale=scale).transpose(1, 2)
+        out.backward(do)
+        dq, dk, dv = O.attention_bwd_ref(q.detach(), k.detach(), v.detach(), do, causal=causal, scale=scale,
+                                         cache_idx=ci)
+        _close(dq, q.grad.numpy(), 1e-10, f"bwd dq {i}")
+        _close(dk, k.grad.numpy(), 1e-10, f"bwd dk {i}")
+        _close(dv, v.grad.numpy(), 1e-10, f"bwd dv {i}")
+
+
+def pin_backward_finite_difference(O):
+    # Central differences of L = sum(out * g) against the analytic gradient
+    # on a few coordinates of q, k and v (second-order accurate).
+    B, N, Hq, Hkv, d, scale = 1, 6, 2, 1, 3, 0.6
+    q = _rand((B, N, Hq, d), 170).numpy()
+    k = _rand((B, N, Hkv, d), 171).numpy()
+    v = _rand((B, N, Hkv, d), 172).numpy()
+    g = _rand((B, N, Hq, d), 173).numpy()
+    dq, dk, dv = O.attention_bwd_ref(q, k, v, g, causal=True, scale=scale)
+
+    def loss(qq, kk, vv):
+        o, _ = O.attention_ref(qq, kk, vv, causal=True, scale=scale)
+        return float(np.sum(o * g))
+
+    eps = 1e-5
+    for arr, grad, name in ((q, dq, "q"), (k, dk, "k"), (v, dv, "v")):
+        for idx in [(0, 1, 0, 0), (0, 3, 0, 2), (0, 5, 0, 1)]:
+            idx = idx if arr.shape[2] > idx[2] else (idx[0], idx[1], 0, idx[3])
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += eps
+            a2[idx] -= eps
+            args1 = {"q": (a1, k, v), "k": (q, a1, v), "v": (q, k, a1)}[name]
+            args2 = {"q": (a2, k, v), "k": (q, a2, v), "v": (q, k, a2)}[name]
+            fd = (loss(*args1) - loss(*args2)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7, f"finite difference d{name}{idx}: {fd} vs {grad[idx]}"
+
+
 ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
-            pin_block_step, pin_lse_merge, pin_schedule]
+            pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference]

@@ -39,6 +39,11 @@ MUTATIONS = [
     ("merge lse drops max", "lse = np.where(has, base + np.log(safe), NEG_INF)", "lse = np.where(has, np.log(safe), NEG_INF)"),
     ("merge unweighted", "out = (w_t * o).sum(axis=0) /", "out = o.sum(axis=0) /"),
     ("softmax base", "w = np.exp(s - base[:, None])", "w = np.exp(s - base[:, None] - 1.0)"),
+    ("bwd D term dropped", "ds = p * (dp - D[:, None])", "ds = p * dp"),
+    ("bwd dv transposed", "dv[b, :, hk, :] += p.T @ do[b, :, h, :]", "dv[b, :, hk, :] += p.T @ q[b, :, h, :]"),
+    ("bwd dk scale dropped", "dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])", "dk[b, :, hk, :] += (ds.T @ q[b, :, h, :])"),
+    ("bwd dq uses v", "dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])", "dq[b, :, h, :] = scale * (ds @ v[b, :, hk, :])"),
+    ("bwd group not summed", "dk[b, :, hk, :] += scale", "dk[b, :, hk, :] = scale"),
 ]
 
 
