@@ -146,6 +146,28 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
               int B, int Hq, int64_t N_q, int d, int out_dtype, void* stream);
 
 /*
+ * ring_attn_bwd -- gradients of ring_attn_fwd (bf16), for training.  The
+ * pages define the forward only (and use it for training: Ring Attention
+ * with FSDP in "Billion-token context window engineering", production
+ * parameters); the backward is the gradient of that definition:
+ *     D_t = dout_t . out_t,  p_tj = exp(scale q_t . k_j - lse_t) on visible pairs,
+ *     ds_tj = p_tj (dout_t . v_j - D_t),
+ *     dq_t = scale sum_j ds_tj k_j,  dk_j = scale sum_t ds_tj q_t,
+ *     dv_j = sum_t p_tj dout_t   (dk, dv summed over a GQA group's heads).
+ * q, out, dout, dq: [B, N_q, Hq, d] bf16; k, v, dk, dv: [B, N_kv, Hkv, d]
+ * bf16; lse: [B, Hq, N_q] float32 as returned by ring_attn_fwd (out too).
+ * causal / cache_idx / scale as in ring_attn_fwd.  Every element of dq, dk
+ * and dv is written (zero for rows with no visible partner).  A stream-
+ * ordered workspace of 2 * B * Hq * ceil(N_q / 128) * 128 floats is
+ * allocated and freed on `stream`.  Returns RA_OK, RA_ERR_INVALID_ARG,
+ * RA_ERR_UNSUPPORTED, RA_ERR_CUDA or RA_ERR_OOM.
+ */
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
+                  int causal, int64_t cache_idx, float scale, void* stream);
+
+/*
  * ring_attn_fwd_noalloc -- ring_attn_fwd for incremental queries
  * (cache_idx >= 0) that allocates no device memory.  The pages have no
  * counterpart; this exists for callers that cannot let a library allocate:

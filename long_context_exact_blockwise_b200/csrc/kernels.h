@@ -77,6 +77,27 @@ cudaError_t launch_finalize(const float* acc, const float* m, const float* l, vo
 cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse,
                              int B, int Hq, long long N_q, int d, int out_f32, cudaStream_t stream);
 
+// Backward pass (bf16 tensors, float32 workspace of 2 * B * Hq * Npad floats).
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* ws_lse2;  // [B, Hq, Npad]
+  float* ws_d;     // [B, Hq, Npad]
+  int B, Hq, Hkv, d;
+  long long N_q, N_kv, Npad;
+  long long q_pos0;
+  int causal;
+  float scale;
+};
+cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t stream);
+
 // y = exp2_poly2(x) elementwise (the FMA-pipe exp2 of the softmax), for tests.
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 

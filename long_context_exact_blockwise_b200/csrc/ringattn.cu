@@ -14,6 +14,7 @@
 // The kernels and their launchers (one translation unit: the status word is
 // shared without relocatable device code).
 #include "fwd_sm100.cuh"
+#include "bwd_sm100.cuh"
 #include "fwd_simt.cuh"
 #include "merge.cuh"
 
@@ -307,6 +308,46 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return finish(launch_lse_merge(o_parts, lse_parts, S, out, lse, B, Hq, N_q, d, out_dtype == RA_DTYPE_F32, st), st,
                 "lse_merge");
+}
+
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
+                  int64_t cache_idx, float scale, void* stream) {
+  if (!dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
+  if (!(aligned16(dout) && aligned16(dq) && aligned16(dk) && aligned16(dv))) return RA_ERR_INVALID_ARG;
+  // Same shape rules as ring_attn_fwd (one chunk spanning the sequence).
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, N_kv, 1, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N_q == 0) return RA_OK;
+  if ((r = check_device(nullptr)) != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long Npad = (N_q + 127) / 128 * 128;
+  const size_t ws_bytes = (size_t)2 * B * Hq * Npad * sizeof(float);
+  if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
+    t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
+    return RA_ERR_OOM;
+  }
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, ws_bytes, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
+    return RA_ERR_OOM;
+  }
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.ws_lse2 = static_cast<float*>(ws);
+  a.ws_d = a.ws_lse2 + (size_t)B * Hq * Npad;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv; a.Npad = Npad;
+  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.causal = causal; a.scale = scale;
+  e = launch_bwd_sm100(a, st);
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
+  return finish(e, st, "ring_attn_bwd");
 }
 
 int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
-    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_block_step", "ring_attn_finalize",
+    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_bwd", "ring_attn_block_step", "ring_attn_finalize",
     "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
@@ -54,6 +54,7 @@ _SIGS = {
     "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
     "ring_attn_block_step": [_p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _i, _p],
     "ring_attn_finalize": [_p, _p, _p, _p, _p, _i, _i, _l, _i, _i, _p],
     "lse_merge": [_p, _p, _i, _p, _p, _i, _i, _l, _i, _i, _p],
@@ -175,6 +176,25 @@ def ring_attn_fwd_noalloc(q, k, v, *, causal: bool, P: int, cache_idx: int, chun
     Pass ``out`` and ``lse`` to avoid allocations on the Python side too."""
     return _fwd(lib.ring_attn_fwd_noalloc, torch.bfloat16, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
                 stream)
+
+
+def ring_attn_bwd(q, k, v, out, dout, lse, *, causal: bool, cache_idx=None, scale: Optional[float] = None,
+                  dq=None, dk=None, dv=None, stream=None):
+    """Gradients (dq, dk, dv) of ring_attn_fwd's output for upstream dout (bf16)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, torch.bfloat16)
+    _need(lse, "lse", torch.float32)
+    B, N_q, Hq, d = q.shape
+    _, N_kv, Hkv, _ = k.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ci = -1 if cache_idx is None else int(cache_idx)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.ring_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                           _ptr(dv), B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)), ci, sc, _stream(stream, q.device))
+    _check(st, "ring_attn_bwd")
+    return dq, dk, dv
 
 
 def ring_attn(q, k, v, *, causal: bool, P: int, cache_idx=None, scale=None, stream=None):
