@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.828749 GB read + 0.258709 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.087458e9, "src": "2e7ad4d545362cff"},
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.830734 GB read + 0.255677 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.086411e9, "src": "d6d6b77a5bb63a09"},
     # profiles/fwd_sm100_decode_Nq1_Nkv65536.md: 1.073881 GB read + 0.007975 GB written.
     "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.081856e9, "src": "2e7ad4d545362cff"},
     # The full-length decode scales the quarter-length capture by its 4x KV
@@ -52,10 +52,16 @@ NCU_TRAFFIC = {
 }
 
 
-def kernel_source_hash() -> str:
+# Sources that do not affect a pass's kernels, left out of its hash.
+_NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh"}, "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh"}}
+
+
+def kernel_source_hash(pass_: str = "fwd") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_exact_blockwise_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if name in _NOT_IN_HASH[pass_]:
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -184,9 +190,22 @@ def run_ours(args, w, rank, world, device):
     ci = None if w.cache_idx < 0 else w.cache_idx
     fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
 
-    def step():
+    if args.pass_ == "bwd":
+        if w.dtype != "bf16":
+            raise SystemExit("--pass bwd needs a bf16 workload")
         fn(q, k, v, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
            stream=stream)
+        g = torch.Generator(device=device).manual_seed(rank_seed(w, rank) + 99)
+        dout = torch.randn(q.shape, generator=g, device=device).to(q.dtype)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def step():
+            R.ring_attn_bwd(q, k, v, out, dout, lse, causal=w.causal, cache_idx=ci, scale=w.scale, dq=dq, dk=dk,
+                            dv=dv, stream=stream)
+    else:
+        def step():
+            fn(q, k, v, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
+               stream=stream)
 
     def barrier():
         if world > 1:
@@ -227,18 +246,33 @@ def run_ours(args, w, rank, world, device):
     hq = q.cpu().pin_memory()
     hk = k.cpu().pin_memory()
     hv = v.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    xq, xk, xv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if args.pass_ == "bwd":
+        # Inputs: q, k, v, out, dout, lse; results: dq, dk, dv.
+        h_in = [hq, hk, hv, out.cpu().pin_memory(), dout.cpu().pin_memory(), lse.cpu().pin_memory()]
+        x_in = [xq, xk, xv, torch.empty_like(out), torch.empty_like(dout), torch.empty_like(lse)]
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        fn(dq, dk, dv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
-           stream=stream)
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+        def e2e_step():
+            for x, h in zip(x_in, h_in):
+                x.copy_(h, non_blocking=True)
+            R.ring_attn_bwd(*x_in, causal=w.causal, cache_idx=ci, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                            stream=stream)
+            for h, x in zip(h_out, (dq, dk, dv)):
+                h.copy_(x, non_blocking=True)
+    else:
+        h_in = [hq, hk, hv]
+        h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
+
+        def e2e_step():
+            xq.copy_(hq, non_blocking=True)
+            xk.copy_(hk, non_blocking=True)
+            xv.copy_(hv, non_blocking=True)
+            fn(xq, xk, xv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out,
+               lse=lse, stream=stream)
+            h_out[0].copy_(out, non_blocking=True)
+            h_out[1].copy_(lse, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(device)
@@ -252,8 +286,8 @@ def run_ours(args, w, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, device)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
-    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = sum(x.numel() * x.element_size() for x in h_out)
     res = dict(ms_total=ms_total, per_launch_ms=per_launch, launches=launches, clocks=clocks.summary(),
                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, host_inputs=(hq, hk, hv))
     return res
@@ -302,6 +336,31 @@ def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
     return flops, elapsed, rows_done, threads
 
 
+def oracle_bwd_sample(w, host_qkv, budget_s: float, seed: int = 0):
+    """Time the float64 gradient oracle on one (batch, KV-head group) of the
+    first n tokens of workload w, n doubling from 256 while the budget lasts.
+    Returns (flops_done, seconds, description, threads)."""
+    import oracle
+    q, k, v = host_qkv
+    G = w.Hq // w.Hkv
+    g = torch.Generator().manual_seed(seed)
+    flops, elapsed, n, done, last = 0.0, 0.0, 256, [], 0.0
+    # Each doubling of n costs about four times the last size.
+    while elapsed + 4.0 * last <= budget_s and n <= min(w.N_q, 1 << 14):
+        qs = q[:1, :n, :G].double()
+        ks, vs = k[:1, :n, :1].double(), v[:1, :n, :1].double()
+        do = torch.randn(qs.shape, generator=g, dtype=torch.float64)
+        t0 = time.perf_counter()
+        oracle.attention_bwd_ref(qs, ks, vs, do, causal=w.causal, scale=w.scale)
+        last = time.perf_counter() - t0
+        elapsed += last
+        pairs = n * (n + 1) / 2 if w.causal else n * n
+        flops += 2.5 * 4.0 * w.d * G * pairs
+        done.append(n)
+        n *= 2
+    return flops, elapsed, done, os.cpu_count()
+
+
 def host_inputs(w):
     return workloads.make_qkv(w, device="cpu")
 
@@ -313,6 +372,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="2", help="workload key: 1..5, 5d1, 5d8 (default 2)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd: the forward pass (default); bwd: the backward pass (dq, dk, dv)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -321,13 +382,17 @@ def main():
         ap.error("--warmup must be >= 3")
 
     w = workloads.CONFIGS[config_key(args.config)]
+    bwd = args.pass_ == "bwd"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     peaks, peak_src = load_peaks()
-    flops = flops_of(w)
+    # The backward's algorithmic work is 2.5x the forward's (five GEMMs of the
+    # forward's size instead of two); the dQ kernel's recomputation of S and
+    # dP is not counted.
+    flops = flops_of(w) * (2.5 if bwd else 1.0)
     config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
               "causal": w.causal, "P": w.P, "chunk": w.chunk, "cache_idx": w.cache_idx, "k_scale": w.k_scale,
               "global_batch": w.B * world, "l2": "inputs larger than the 126 MB L2, no flush"
@@ -338,6 +403,23 @@ def main():
         if rank != 0:
             return
         hq = host_inputs(w)
+        if bwd:
+            budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+            tot_f, tot_s, sizes = 0.0, 0.0, []
+            for i in range(args.steps):
+                f_, s_, n_, threads = oracle_bwd_sample(w, hq, budget, seed=i + 1)
+                tot_f, tot_s, sizes = tot_f + f_, tot_s + s_, sizes + n_
+            val = tot_f / tot_s / 1e12
+            line = {"impl": "reference", "metric": "attention bwd TFLOP/s", "value": val, "unit": "TFLOP/s",
+                    "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": 1e3 * flops / (val * 1e12), "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                    "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                     "sample": f"float64 gradient oracle on one KV-head group of the first "
+                                               f"n tokens, n in {sorted(set(sizes))}, {tot_s:.1f} s"},
+                    "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+            return
         budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
         for _ in range(args.warmup):
             oracle_sample(w, hq, budget / 4)
@@ -380,22 +462,27 @@ def main():
         bound, unit = "alu", "TFLOP/s"
         # FP32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock.
         peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
-    elif w.cache_idx >= 0 and w.N_q * (w.Hq // w.Hkv) <= 64:
+    elif not bwd and w.cache_idx >= 0 and w.N_q * (w.Hq // w.Hkv) <= 64:
         bound, unit = "hbm", "GB/s"
         achieved = hbm_bytes_of(w) / (launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
-    src_hash = kernel_source_hash()
-    tr = NCU_TRAFFIC.get(w.name)
+    src_hash = kernel_source_hash(args.pass_)
+    tr = NCU_TRAFFIC.get(w.name + (" bwd" if bwd else ""))
     traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and bwd:
+        f_, s_, n_, threads = oracle_bwd_sample(w, tuple(x.cpu() for x in res["host_inputs"]), args.cpu_budget)
+        cpu = {"value": f_ / s_ / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"float64 gradient oracle on one KV-head group of the first n tokens of this "
+                         f"workload, n in {n_}, {s_:.1f} s on the host"}
+    elif rank == 0 and not args.no_cpu_baseline:
         f_, s_, r_, threads = oracle_sample(w, tuple(x.cpu() for x in res["host_inputs"]), args.cpu_budget)
         cpu = {"value": f_ / s_ / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{r_} random (row, head) query rows in runs of 16 of this workload, {s_:.1f} s of "
                          f"float64 oracle work on the host"}
     e2e_val = aggregate_tflops(flops, world, res["e2e_ms"])
     line = {
-        "metric": "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": "attention bwd TFLOP/s" if bwd else "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config,
         "tokens_per_s": w.B * w.N_q * world / (ms_step * 1e-3),
@@ -404,7 +491,8 @@ def main():
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} ({peak_kind if bound == 'tensor' else bound})",
-                     "kernel": "fwd_sm100_kernel" if w.dtype == "bf16" else "simt_attn_kernel",
+                     "kernel": ("bwd_prep + bwd_dkdv + bwd_dq (whole step)" if bwd else
+                                "fwd_sm100_kernel" if w.dtype == "bf16" else "simt_attn_kernel"),
                      "algorithmic_per_launch": flops if unit == "TFLOP/s" else hbm_bytes_of(w)},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],

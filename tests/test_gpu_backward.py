@@ -70,3 +70,19 @@ def test_backward_rejects_bad_arguments():
     with pytest.raises(R.RingAttnError) as ei:
         R.ring_attn_bwd(q, q, q, q, q, lse, causal=True)
     assert ei.value.status == R.RA_ERR_INVALID_ARG
+
+
+def test_backward_medium_size():
+    # 16 query tiles x 16 key tiles per head, causal, GQA 2.
+    R = ra()
+    w = workloads.small(B=1, Hq=4, Hkv=2, N_q=2048, d=128, causal=True, P=1, seed=77)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(78)
+    dout = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    out, lse = R.ring_attn_fwd(q, k, v, causal=True, P=1, scale=w.scale)
+    dq, dk, dv = R.ring_attn_bwd(q, k, v, out, dout, lse, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=True, scale=w.scale)
+    _check(dv, rv, "dv")
+    _check(dk, rk, "dk")
+    _check(dq, rq, "dq")
