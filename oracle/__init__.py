@@ -29,10 +29,12 @@ routine, brute force, closed forms, invariants, the pages' printed schedule).
 from .attention import (
     attention_bwd_ref,
     attention_ref,
+    block_step_bwd_ref,
     block_step_ref,
     finalize_ref,
     init_state,
     lse_merge_ref,
+    ring_bwd_ref,
     ring_ref,
     ring_visit_chunk,
     query_home_chunk,
@@ -41,10 +43,12 @@ from .attention import (
 __all__ = [
     "attention_bwd_ref",
     "attention_ref",
+    "block_step_bwd_ref",
     "block_step_ref",
     "finalize_ref",
     "init_state",
     "lse_merge_ref",
+    "ring_bwd_ref",
     "ring_ref",
     "ring_visit_chunk",
     "query_home_chunk",

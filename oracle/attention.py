@@ -320,3 +320,84 @@ def attention_bwd_ref(q, k, v, dout, *, causal: bool, scale: float, cache_idx: i
             dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
             dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
     return dq, dk, dv
+
+
+def block_step_bwd_ref(q_chunk, k_chunk, v_chunk, dout_chunk, lse_chunk, delta_chunk, q_off: int, k_off: int,
+                       dq, dk, dv, *, causal: bool, scale: float):
+    """Fold one ring visit's share of the gradients into (dq, dk, dv).
+
+    The backward of a ring visit: a query chunk (q, dout, its final lse and
+    delta = rowsum(dout * out), all for the whole sequence's softmax)
+    against one KV chunk.  With p_tj = exp(s_tj - lse_t) on the visible pairs
+    of this visit (s_tj = scale * q_t . k_j, positions q_off + t and k_off + j)
+    and zero elsewhere, every term of attention_bwd_ref that involves only
+    this visit's keys is added:
+        dv_j += sum_t p_tj dout_t
+        ds_tj = p_tj (dout_t . v_j - delta_t)
+        dq_t += scale * sum_j ds_tj k_j
+        dk_j += scale * sum_t ds_tj q_t
+    (dk, dv summed over the query heads of a GQA group).  Summed over all
+    visits this is the full gradient, because p_tj and ds_tj depend on the
+    other chunks only through lse_t and delta_t.
+
+    q_chunk, dout_chunk, dq: [B, Lq, Hq, d]; k_chunk, v_chunk, dk, dv:
+    [B, Lk, Hkv, d]; lse_chunk, delta_chunk: [B, Hq, Lq].  Rows with
+    lse = -inf (no visible key anywhere) contribute nothing.  Returns new
+    (dq, dk, dv); the inputs are not modified.
+    """
+    q, kc, vc, do = _f64(q_chunk), _f64(k_chunk), _f64(v_chunk), _f64(dout_chunk)
+    lse, delta = _f64(lse_chunk), _f64(delta_chunk)
+    dq, dk, dv = (np.array(_f64(x), copy=True) for x in (dq, dk, dv))
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = kc.shape[1], kc.shape[2]
+    vis = _visible(q_off + np.arange(Lq, dtype=np.int64),
+                   k_off + np.arange(Lk, dtype=np.int64), causal)
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            s = scale * (q[b, :, h, :] @ kc[b, :, hk, :].T)
+            live = vis & np.isfinite(lse[b, h])[:, None]
+            base = np.where(np.isfinite(lse[b, h]), lse[b, h], 0.0)
+            p = np.where(live, np.exp(np.where(live, s, 0.0) - base[:, None]), 0.0)
+            dp = do[b, :, h, :] @ vc[b, :, hk, :].T
+            ds = p * (dp - delta[b, h][:, None])
+            dv[b, :, hk, :] += p.T @ do[b, :, h, :]
+            dq[b, :, h, :] += scale * (ds @ kc[b, :, hk, :])
+            dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
+    return dq, dk, dv
+
+
+def ring_bwd_ref(q, k, v, dout, *, causal: bool, scale: float, P: int, order="forward"):
+    """The backward emulated as a ring: query chunk i visits every KV chunk.
+
+    The forward (out, lse) comes from attention_ref; delta = rowsum(dout *
+    out).  Query chunk i visits KV chunks in ring order; its dq accumulates
+    locally, while the (dk, dv) accumulators of each KV chunk gather one
+    visit's share from every query chunk (in the ring they travel with the
+    chunk).  Square causal prefill or non-causal, N divisible by P.  Returns
+    (dq, dk, dv) in the layouts of attention_bwd_ref.
+    """
+    q64, k64, v64, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, Hq, d = q64.shape
+    if k64.shape[1] != N or N % P != 0:
+        raise ValueError("ring_bwd_ref needs N_q == N_kv divisible by P")
+    L = N // P
+    out, lse = attention_ref(q64, k64, v64, causal=causal, scale=scale)
+    delta = np.einsum("bthe,bthe->bht", do, out)
+    dq = np.zeros_like(q64)
+    dk = np.zeros_like(k64)
+    dv = np.zeros_like(v64)
+    for i in range(P):
+        qs = slice(i * L, (i + 1) * L)
+        for s in range(P):
+            if order == "forward":
+                j = ring_visit_chunk(i, s, P, 1)
+            elif order == "backward":
+                j = ring_visit_chunk(i, s, P, -1)
+            else:
+                j = int(order[i][s])
+            ks = slice(j * L, (j + 1) * L)
+            dq[:, qs], dk[:, ks], dv[:, ks] = block_step_bwd_ref(
+                q64[:, qs], k64[:, ks], v64[:, ks], do[:, qs], lse[:, :, qs], delta[:, :, qs], i * L, j * L,
+                dq[:, qs], dk[:, ks], dv[:, ks], causal=causal, scale=scale)
+    return dq, dk, dv

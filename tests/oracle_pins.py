@@ -368,5 +368,46 @@ def pin_backward_finite_difference(O):
             assert abs(fd - grad[idx]) <= 1e-7, f"finite difference d{name}{idx}: {fd} vs {grad[idx]}"
 
 
+def _autograd_grads(q, k, v, do, causal, scale):
+    """Gradients by torch autograd through float64 SDPA (GQA by repeated heads)."""
+    q, k, v = (x.clone().requires_grad_(True) for x in (q, k, v))
+    G = q.shape[2] // k.shape[2]
+    N_q, N_kv = q.shape[1], k.shape[1]
+    mask = (torch.arange(N_kv)[None, :] <= torch.arange(N_q)[:, None]) if causal else \
+        torch.ones(N_q, N_kv, dtype=torch.bool)
+    out = F.scaled_dot_product_attention(q.transpose(1, 2), k.repeat_interleave(G, dim=2).transpose(1, 2),
+                                         v.repeat_interleave(G, dim=2).transpose(1, 2), attn_mask=mask,
+                                         scale=scale).transpose(1, 2)
+    out.backward(do)
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+def pin_backward_ring(O):
+    # The ring backward (block_step_bwd_ref over every (query chunk, KV
+    # chunk) visit, in ring order, forward, backward or a random order per
+    # query chunk) against torch autograd of the whole-sequence attention.
+    rng = np.random.default_rng(7)
+    cases = [(2, 12, 4, 2, 8, True, 0.3), (1, 12, 2, 2, 4, False, 0.7), (1, 10, 4, 1, 8, True, 0.45)]
+    for i, (B, N, Hq, Hkv, d, causal, scale) in enumerate(cases):
+        q = _rand((B, N, Hq, d), 180 + i)
+        k = _rand((B, N, Hkv, d), 190 + i)
+        v = _rand((B, N, Hkv, d), 200 + i)
+        do = _rand((B, N, Hq, d), 210 + i)
+        ref = _autograd_grads(q, k, v, do, causal, scale)
+        for P in [x for x in (1, 2, 3, 4, 5) if N % x == 0]:
+            perm = [list(rng.permutation(P)) for _ in range(P)]
+            for order in ("forward", "backward", perm):
+                got = O.ring_bwd_ref(q, k, v, do, causal=causal, scale=scale, P=P, order=order)
+                for g, r, name in zip(got, ref, ("dq", "dk", "dv")):
+                    _close(g, r, 1e-10, f"ring bwd {name} case {i} P={P} order={order}")
+    # A visit whose keys all lie in the future of every query adds nothing.
+    q, k, v, do = (_rand((1, 4, 2, 4), 220 + j) for j in range(4))
+    lse = np.zeros((1, 2, 4))
+    z = np.zeros((1, 4, 2, 4))
+    dq, dk, dv = O.block_step_bwd_ref(q, k, v, do, lse, lse, 0, 4, z, z, z, causal=True, scale=0.5)
+    assert not (dq.any() or dk.any() or dv.any()), "a fully masked backward visit changed the gradients"
+
+
 ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
-            pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference]
+            pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference,
+            pin_backward_ring]

@@ -44,6 +44,16 @@ MUTATIONS = [
     ("bwd dk scale dropped", "dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])", "dk[b, :, hk, :] += (ds.T @ q[b, :, h, :])"),
     ("bwd dq uses v", "dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])", "dq[b, :, h, :] = scale * (ds @ v[b, :, hk, :])"),
     ("bwd group not summed", "dk[b, :, hk, :] += scale", "dk[b, :, hk, :] = scale"),
+    ("bwd visit drops delta", "ds = p * (dp - delta[b, h][:, None])", "ds = p * dp"),
+    ("bwd visit lse sign", "np.exp(np.where(live, s, 0.0) - base[:, None])",
+     "np.exp(np.where(live, s, 0.0) + base[:, None])"),
+    ("bwd visit dq unscaled", "dq[b, :, h, :] += scale * (ds @ kc[b, :, hk, :])",
+     "dq[b, :, h, :] += (ds @ kc[b, :, hk, :])"),
+    ("bwd visit dq overwritten", "dq[b, :, h, :] += scale * (ds @ kc[b, :, hk, :])",
+     "dq[b, :, h, :] = scale * (ds @ kc[b, :, hk, :])"),
+    ("bwd ring wrong kv chunk", "ks = slice(j * L, (j + 1) * L)", "ks = slice(i * L, (i + 1) * L)"),
+    ("bwd visit dk from dout", "dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])",
+     "dk[b, :, hk, :] += scale * (ds.T @ do[b, :, h, :])"),
 ]
 
 
