@@ -28,9 +28,11 @@ routine, brute force, closed forms, invariants, the pages' printed schedule).
 """
 from .attention import (
     attention_bwd_ref,
+    attention_fp8kv_ref,
     attention_ref,
     block_step_bwd_ref,
     block_step_ref,
+    decode_e4m3,
     finalize_ref,
     init_state,
     lse_merge_ref,
@@ -42,9 +44,11 @@ from .attention import (
 
 __all__ = [
     "attention_bwd_ref",
+    "attention_fp8kv_ref",
     "attention_ref",
     "block_step_bwd_ref",
     "block_step_ref",
+    "decode_e4m3",
     "finalize_ref",
     "init_state",
     "lse_merge_ref",

@@ -401,3 +401,47 @@ def ring_bwd_ref(q, k, v, dout, *, causal: bool, scale: float, P: int, order="fo
                 q64[:, qs], k64[:, ks], v64[:, ks], do[:, qs], lse[:, :, qs], delta[:, :, qs], i * L, j * L,
                 dq[:, qs], dk[:, ks], dv[:, ks], causal=causal, scale=scale)
     return dq, dk, dv
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """FP8 E4M3 codes (uint8) to float64, from the format's definition.
+
+    Bit 7 is the sign, bits 6..3 the exponent field e (bias 7), bits 2..0 the
+    mantissa m.  e = 0: subnormal, (-1)^s * 2^-6 * m/8.  e = 15 with m = 7:
+    NaN (the format has no infinities).  Otherwise (-1)^s * 2^(e-7) * (1 + m/8).
+    The largest finite magnitude is 448.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def attention_fp8kv_ref(q, k8, v8, k_scale, v_scale, *, causal: bool, scale: float, cache_idx: int = -1):
+    """Attention over an FP8 (E4M3) KV cache with per-(batch, KV head) scales.
+
+    The pages ask for a quantised KV cache in serving ("Billion-token context
+    window engineering", production parameters: 4-/8-bit KV quantisation;
+    "RingAttention vs RAG" §2.3: FP8 deployment; "From hundreds of
+    milliseconds to a million tokens", KV-cache compression by quantisation).
+    The cache holds codes k8, v8 [B, N_kv, Hkv, d] (uint8) and float32 scales
+    k_scale, v_scale [B, Hkv]; the keys and values it stands for are
+        k[b, j, h, :] = decode_e4m3(k8[b, j, h, :]) * k_scale[b, h]
+    (likewise v), and the result is exact attention (attention_ref) over
+    those dequantised keys and values.  Returns (out, lse) as attention_ref.
+    """
+    ks = np.asarray(_f64(k_scale))
+    vs = np.asarray(_f64(v_scale))
+    k = decode_e4m3(_u8(k8)) * ks[:, None, :, None]
+    v = decode_e4m3(_u8(v8)) * vs[:, None, :, None]
+    return attention_ref(q, k, v, causal=causal, scale=scale, cache_idx=cache_idx)
+
+
+def _u8(x) -> np.ndarray:
+    """uint8 codes from a torch tensor (any device) or array."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.asarray(x, dtype=np.uint8)

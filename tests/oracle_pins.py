@@ -408,6 +408,51 @@ def pin_backward_ring(O):
     assert not (dq.any() or dk.any() or dv.any()), "a fully masked backward visit changed the gradients"
 
 
+def pin_fp8_decode(O):
+    # Every E4M3 code against torch's float8_e4m3fn (a library decoder), and
+    # values fixed by the format: 1.0, the largest finite 448, the smallest
+    # subnormal 2^-9, the smallest normal 2^-6, signed zero, NaN.
+    codes = np.arange(256, dtype=np.uint8)
+    got = O.decode_e4m3(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(lib)), "E4M3 NaN codes differ from the library"
+    fin = ~np.isnan(lib)
+    assert np.array_equal(got[fin], lib[fin]), "E4M3 decode differs from the library"
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(lib[fin])), "E4M3 sign of zero differs"
+    fixed = {0x38: 1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x08: 2.0 ** -6, 0xB8: -1.0, 0x3C: 1.5, 0x00: 0.0}
+    for c, v in fixed.items():
+        assert O.decode_e4m3(np.array([c], dtype=np.uint8))[0] == v, hex(c)
+    assert np.isnan(O.decode_e4m3(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def pin_fp8kv_attention(O):
+    # Attention over an FP8 cache against torch float64 SDPA on keys and values
+    # dequantised through torch's own float8 type (GQA by repeated heads,
+    # cache_idx by an explicit mask), plus the scale identities.
+    B, N_q, N_kv, Hq, Hkv, d, ci, scale = 2, 5, 40, 4, 2, 8, 35, 0.4
+    rng = np.random.default_rng(3)
+    q = torch.from_numpy(rng.standard_normal((B, N_q, Hq, d)))
+    k8 = torch.from_numpy(rng.integers(0, 256, (B, N_kv, Hkv, d), dtype=np.uint8))
+    v8 = torch.from_numpy(rng.integers(0, 256, (B, N_kv, Hkv, d), dtype=np.uint8))
+    # Keep the codes finite (0x7f / 0xff are NaN) and the logits moderate.
+    k8 = torch.where((k8 & 0x7F) >= 0x70, k8 & 0xB7, k8)
+    v8 = torch.where((v8 & 0x7F) == 0x7F, v8 & 0xF7, v8)
+    ks = torch.tensor([[0.003, 0.005], [0.004, 0.002]], dtype=torch.float64)
+    vs = torch.tensor([[0.02, 0.01], [0.03, 0.015]], dtype=torch.float64)
+    out, lse = O.attention_fp8kv_ref(q, k8, v8, ks, vs, causal=True, scale=scale, cache_idx=ci)
+    kd = k8.view(torch.float8_e4m3fn).to(torch.float64) * ks[:, None, :, None]
+    vd = v8.view(torch.float8_e4m3fn).to(torch.float64) * vs[:, None, :, None]
+    ro, rl = _sdpa_case(q, kd, vd, True, scale, ci)
+    _close(out, ro, TOL, "fp8kv out vs sdpa")
+    _close(lse, rl, TOL, "fp8kv lse vs sdpa")
+    o2, l2 = O.attention_fp8kv_ref(q / 2, k8, v8, ks * 2, vs, causal=True, scale=scale, cache_idx=ci)
+    _close(o2, out, 1e-12, "k_scale x2 with q / 2")
+    _close(l2, lse, 1e-12, "k_scale x2 with q / 2 (lse)")
+    o3, l3 = O.attention_fp8kv_ref(q, k8, v8, ks, vs * 2, causal=True, scale=scale, cache_idx=ci)
+    _close(o3, 2 * out, 1e-12, "v_scale x2 doubles out")
+    _close(l3, lse, 1e-12, "v_scale leaves lse")
+
+
 ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
             pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference,
-            pin_backward_ring]
+            pin_backward_ring, pin_fp8_decode, pin_fp8kv_attention]

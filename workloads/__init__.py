@@ -22,7 +22,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["Workload", "CONFIGS", "make_qkv", "workload", "small"]
+__all__ = ["Workload", "CONFIGS", "make_qkv", "make_fp8_kv", "workload", "small"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -43,6 +43,7 @@ class Workload:
     cache_idx: int = -1   # -1: plain prefill (N_q == N_kv); >= 0: queries sit at cache_idx + t
     k_scale: float = 1.0  # exact power-of-two multiplier applied to K before the cast
     seed: int = 0         # q uses seed, k seed+1, v seed+2
+    kv_dtype: str = "bf16"  # "fp8": the KV cache is stored as FP8 E4M3 codes with scales (make_fp8_kv)
 
     @property
     def scale(self) -> float:
@@ -75,6 +76,13 @@ CONFIGS = {
                     dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5200),
     # A quarter-length decode cache (1.07 GB of K/V, still 8x the L2) for
     # profiler captures that must stay small.
+    # The full-length decode with its KV cache stored as FP8 E4M3 codes.
+    "5d1f8": Workload("cache_idx_decode_fp8kv_Nq1_Nkv262144", B=4, Hq=32, Hkv=8, N_q=1, N_kv=262144, d=128,
+                      dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 1, seed=5400,
+                      kv_dtype="fp8"),
+    "5d8f8": Workload("cache_idx_decode_fp8kv_Nq8_Nkv262144", B=4, Hq=32, Hkv=8, N_q=8, N_kv=262144, d=128,
+                      dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5500,
+                      kv_dtype="fp8"),
     "5d1s": Workload("cache_idx_decode_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
                      dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5300),
 }
@@ -85,7 +93,7 @@ def workload(key) -> Workload:
 
 
 def small(B=1, Hq=2, Hkv=1, N_q=200, N_kv=None, d=64, dtype="bf16", causal=True, P=2,
-          chunk=None, cache_idx=-1, k_scale=1.0, seed=7, name="small") -> Workload:
+          chunk=None, cache_idx=-1, k_scale=1.0, seed=7, name="small", kv_dtype="bf16") -> Workload:
     """A small problem for parity tests (sizes the CPU oracle finishes quickly)."""
     if N_kv is None:
         N_kv = N_q if cache_idx < 0 else cache_idx + N_q
@@ -93,7 +101,7 @@ def small(B=1, Hq=2, Hkv=1, N_q=200, N_kv=None, d=64, dtype="bf16", causal=True,
         chunk = N_kv // P
     return Workload(name, B=B, Hq=Hq, Hkv=Hkv, N_q=N_q, N_kv=N_kv, d=d, dtype=dtype,
                     causal=causal, P=P, chunk=chunk, cache_idx=cache_idx, k_scale=k_scale,
-                    seed=seed)
+                    seed=seed, kv_dtype=kv_dtype)
 
 
 def _randn(shape, seed: int, device, mult: float, dtype: torch.dtype) -> torch.Tensor:
@@ -113,3 +121,31 @@ def make_qkv(w: Workload, device="cpu", seed: Optional[int] = None):
     k = _randn((w.B, w.N_kv, w.Hkv, w.d), s + 1, device, w.k_scale, dt)
     v = _randn((w.B, w.N_kv, w.Hkv, w.d), s + 2, device, 1.0, dt)
     return q, k, v
+
+
+E4M3_MAX = 448.0  # largest finite FP8 E4M3 magnitude
+
+
+def make_fp8_kv(w: Workload, device="cpu", seed: Optional[int] = None):
+    """Return (q, k8, v8, k_scale, v_scale) for workload ``w``: an FP8 KV cache.
+
+    q is drawn as in make_qkv.  K and V are drawn as float32 exactly as
+    make_qkv draws them, then quantised per (batch, KV head): scale =
+    amax / 448 over that head's tokens and channels (1 where the head is all
+    zero), codes = round-to-nearest-even of x / scale to FP8 E4M3 (torch's
+    float8_e4m3fn cast).  k8, v8 are the codes as uint8 [B, N_kv, Hkv, d];
+    k_scale, v_scale are float32 [B, Hkv].  This is input preparation only:
+    the codes and scales are the cache both sides read.
+    """
+    s = w.seed if seed is None else seed
+    q = _randn((w.B, w.N_q, w.Hq, w.d), s + 0, device, 1.0, w.torch_dtype)
+    out = [q]
+    scales = []
+    for off, mult in ((1, w.k_scale), (2, 1.0)):
+        x = _randn((w.B, w.N_kv, w.Hkv, w.d), s + off, device, mult, torch.float32)
+        amax = x.abs().amax(dim=(1, 3))                      # [B, Hkv]
+        sc = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+        codes = (x / sc[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        out.append(codes.contiguous())
+        scales.append(sc.contiguous())
+    return out[0], out[1], out[2], scales[0], scales[1]
