@@ -411,13 +411,15 @@ def decode_e4m3(codes) -> np.ndarray:
     NaN (the format has no infinities).  Otherwise (-1)^s * 2^(e-7) * (1 + m/8).
     The largest finite magnitude is 448.
     """
-    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    # The definition is applied to the 256 codes once; arrays of codes then
+    # index that table.
+    c = np.arange(256, dtype=np.int64)
     sign = np.where((c >> 7) & 1, -1.0, 1.0)
     e = (c >> 3) & 0xF
     m = (c & 0x7).astype(np.float64)
     mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
     mag = np.where((e == 15) & (m == 7), np.nan, mag)
-    return sign * mag
+    return (sign * mag)[np.asarray(codes, dtype=np.uint8)]
 
 
 def attention_fp8kv_ref(q, k8, v8, k_scale, v_scale, *, causal: bool, scale: float, cache_idx: int = -1):

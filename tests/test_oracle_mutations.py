@@ -54,7 +54,7 @@ MUTATIONS = [
     ("bwd ring wrong kv chunk", "ks = slice(j * L, (j + 1) * L)", "ks = slice(i * L, (i + 1) * L)"),
     ("e4m3 exponent bias 8", "np.ldexp(1.0 + m / 8.0, e - 7)", "np.ldexp(1.0 + m / 8.0, e - 8)"),
     ("e4m3 subnormal as 2^-7", "np.ldexp(m / 8.0, -6)", "np.ldexp(m / 8.0, -7)"),
-    ("e4m3 sign dropped", "return sign * mag", "return mag"),
+    ("e4m3 sign dropped", "return (sign * mag)[", "return (mag)["),
     ("e4m3 mantissa step 1/16", "(1.0 + m / 8.0, e - 7)", "(1.0 + m / 16.0, e - 7)"),
     ("fp8 v scaled by k_scale", "v = decode_e4m3(_u8(v8)) * vs[", "v = decode_e4m3(_u8(v8)) * ks["),
     ("fp8 scale transposed", "k = decode_e4m3(_u8(k8)) * ks[:, None, :, None]",
