@@ -95,9 +95,12 @@ def flops_of(w: workloads.Workload) -> float:
 
 
 def hbm_bytes_of(w: workloads.Workload) -> float:
-    """Minimum HBM traffic: q, k, v read once, out written once, lse written."""
+    """Minimum HBM traffic: q, k, v read once, out written once, lse written
+    (an FP8 cache: one byte per K/V element plus its scales)."""
     es = 2 if w.dtype == "bf16" else 4
-    return es * (2 * w.B * w.N_q * w.Hq * w.d + 2 * w.B * w.N_kv * w.Hkv * w.d) + 4 * w.B * w.Hq * w.N_q
+    kv_es = 1 if w.kv_dtype == "fp8" else es
+    kv = kv_es * 2 * w.B * w.N_kv * w.Hkv * w.d + (8 * w.B * w.Hkv if w.kv_dtype == "fp8" else 0)
+    return es * 2 * w.B * w.N_q * w.Hq * w.d + kv + 4 * w.B * w.Hq * w.N_q
 
 
 # ----------------------------------------------------------------- ranks
@@ -184,15 +187,23 @@ def run_ours(args, w, rank, world, device):
 
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    q, k, v = workloads.make_qkv(w, device=device, seed=rank_seed(w, rank))
+    fp8 = w.kv_dtype == "fp8"
+    if fp8:
+        q, k, v, k_sc, v_sc = workloads.make_fp8_kv(w, device=device, seed=rank_seed(w, rank))
+    else:
+        q, k, v = workloads.make_qkv(w, device=device, seed=rank_seed(w, rank))
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.N_q), device=device, dtype=torch.float32)
     ci = None if w.cache_idx < 0 else w.cache_idx
-    fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
+    if fp8:
+        def fn(q_, k_, v_, **kw):
+            return R.ring_attn_fwd_fp8kv(q_, k_, v_, k_sc, v_sc, **kw)
+    else:
+        fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
 
     if args.pass_ == "bwd":
-        if w.dtype != "bf16":
-            raise SystemExit("--pass bwd needs a bf16 workload")
+        if w.dtype != "bf16" or fp8:
+            raise SystemExit("--pass bwd needs a bf16 workload with a bf16 KV cache")
         fn(q, k, v, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out, lse=lse,
            stream=stream)
         g = torch.Generator(device=device).manual_seed(rank_seed(w, rank) + 99)
@@ -265,10 +276,17 @@ def run_ours(args, w, rank, world, device):
         h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
                  torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
 
+        if fp8:
+            h_sc = [k_sc.cpu().pin_memory(), v_sc.cpu().pin_memory()]
+            x_sc = [k_sc, v_sc]  # the call reads the scales from these device tensors
+
         def e2e_step():
             xq.copy_(hq, non_blocking=True)
             xk.copy_(hk, non_blocking=True)
             xv.copy_(hv, non_blocking=True)
+            if fp8:
+                for x, h in zip(x_sc, h_sc):
+                    x.copy_(h, non_blocking=True)
             fn(xq, xk, xv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out,
                lse=lse, stream=stream)
             h_out[0].copy_(out, non_blocking=True)
@@ -286,10 +304,11 @@ def run_ours(args, w, rank, world, device):
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, device)
-    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    h2d = sum(x.numel() * x.element_size() for x in h_in) + (16 * w.B * w.Hkv if fp8 else 0)
     d2h = sum(x.numel() * x.element_size() for x in h_out)
     res = dict(ms_total=ms_total, per_launch_ms=per_launch, launches=launches, clocks=clocks.summary(),
-               e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, host_inputs=(hq, hk, hv))
+               e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+               host_inputs=(hq, hk, hv) + ((k_sc.cpu(), v_sc.cpu()) if fp8 else ()))
     return res
 
 
@@ -303,10 +322,21 @@ def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
         from threadpoolctl import threadpool_info
     except Exception:  # pragma: no cover
         threadpool_info = None
-    q, k, v = host_qkv
+    q, k, v = host_qkv[:3]
     rng = np.random.default_rng(seed)
     G = w.Hq // w.Hkv
     kf = {}
+    if w.kv_dtype == "fp8":
+        # Dequantise one KV head of the FP8 cache by the oracle's decoder.
+        k_sc, v_sc = (x.double().numpy() for x in host_qkv[3:5])
+
+        def kv_head(hk):
+            dk = oracle.decode_e4m3(k[:, :, hk:hk + 1].numpy()) * k_sc[:, None, hk:hk + 1, None]
+            dv = oracle.decode_e4m3(v[:, :, hk:hk + 1].numpy()) * v_sc[:, None, hk:hk + 1, None]
+            return dk, dv
+    else:
+        def kv_head(hk):
+            return k[:, :, hk:hk + 1].double().numpy(), v[:, :, hk:hk + 1].double().numpy()
     flops = 0.0
     rows_done = 0
     t_start = time.perf_counter()
@@ -315,7 +345,7 @@ def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
         h = int(rng.integers(0, w.Hq))
         hk = h // G
         if hk not in kf:
-            kf[hk] = (k[:, :, hk:hk + 1].double().numpy(), v[:, :, hk:hk + 1].double().numpy())
+            kf[hk] = kv_head(hk)
         r0 = int(rng.integers(0, max(1, w.N_q - 16)))
         nr = min(16, w.N_q - r0)
         qs = q[:, r0:r0 + nr, h:h + 1].double().numpy()
@@ -362,6 +392,8 @@ def oracle_bwd_sample(w, host_qkv, budget_s: float, seed: int = 0):
 
 
 def host_inputs(w):
+    if w.kv_dtype == "fp8":
+        return workloads.make_fp8_kv(w, device="cpu")
     return workloads.make_qkv(w, device="cpu")
 
 
@@ -393,7 +425,8 @@ def main():
     # forward's size instead of two); the dQ kernel's recomputation of S and
     # dP is not counted.
     flops = flops_of(w) * (2.5 if bwd else 1.0)
-    config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
+    config = {"workload": w.name, "kv_cache": "fp8 e4m3 + per-head scales" if w.kv_dtype == "fp8" else w.dtype,
+              "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
               "causal": w.causal, "P": w.P, "chunk": w.chunk, "cache_idx": w.cache_idx, "k_scale": w.k_scale,
               "global_batch": w.B * world, "l2": "inputs larger than the 126 MB L2, no flush"
               if hbm_bytes_of(w) > 126e6 else "inputs fit in L2 (small correctness case)",
@@ -492,6 +525,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} ({peak_kind if bound == 'tensor' else bound})",
                      "kernel": ("bwd_prep + bwd_dkdv + bwd_dq (whole step)" if bwd else
+                                "fwd_sm100_kernel (FP8 KV, converter warpgroup)" if w.kv_dtype == "fp8" else
                                 "fwd_sm100_kernel" if w.dtype == "bf16" else "simt_attn_kernel"),
                      "algorithmic_per_launch": flops if unit == "TFLOP/s" else hbm_bytes_of(w)},
         "cpu_baseline": cpu,

@@ -168,6 +168,55 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
                   int causal, int64_t cache_idx, float scale, void* stream);
 
 /*
+ * ring_attn_fwd_fp8kv -- ring_attn_fwd over a KV cache stored as FP8 E4M3
+ * codes (the pages' quantised KV cache for serving: "Billion-token context
+ * window engineering", production parameters; "RingAttention vs RAG" §2.3;
+ * "From hundreds of milliseconds to a million tokens", KV-cache
+ * compression).  k8, v8: [B, N_kv, Hkv, d] E4M3 codes (one byte each);
+ * k_scale, v_scale: [B, Hkv] float32.  The keys and values attended to are
+ *     k[b, j, h, :] = e4m3(k8[b, j, h, :]) * k_scale[b, h]   (v likewise),
+ * and out / lse are exact attention over them, as ring_attn_fwd computes
+ * them (q, out bf16; lse float32; same shapes, causal, chunk, P, cache_idx
+ * and scale rules; incremental queries use split-KV partials and a stream-
+ * ordered workspace).  The tensor cores read the codes decoded to bf16,
+ * which is exact for every E4M3 value.  All pointers are device memory
+ * owned by the caller; q, k8, v8, out 16-byte aligned.  Returns RA_OK,
+ * RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA or RA_ERR_OOM.
+ */
+int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const float* k_scale,
+                        const float* v_scale, void* out, float* lse, int B, int Hq, int Hkv,
+                        int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P,
+                        int64_t cache_idx, float scale, void* stream);
+
+/*
+ * ring_attn_bwd_block_step -- the backward of one ring visit: adds, in
+ * place, the share of dq, dk, dv that comes from the pairs of query chunk
+ * q_chunk [B, Lq, Hq, d] (global positions q_off + t) and KV chunk
+ * k_chunk / v_chunk [B, Lk, Hkv, d] (positions k_off + j).  With the query
+ * rows' final lse (over the whole sequence, as ring_attn_finalize or
+ * ring_attn_fwd return it) and D_t = dout_t . out_t:
+ *     p_tj = exp(scale q_t . k_j - lse_t)       on visible pairs, else 0
+ *     ds_tj = p_tj (dout_t . v_j - D_t)
+ *     dq_acc_t += scale sum_j ds_tj k_j
+ *     dk_acc_j += scale sum_t ds_tj q_t,   dv_acc_j += sum_t p_tj dout_t
+ * (dk, dv summed over a GQA group's heads).  Summed over every visit of a
+ * ring this is ring_attn_bwd's result: the gradient of the Ring Attention
+ * page's blockwise loop (§3.1), whose dk / dv travel with their KV chunk.
+ * q/k/v/out/dout chunks bf16 (out_chunk and dout_chunk [B, Lq, Hq, d]);
+ * lse_chunk [B, Hq, Lq] float32; dq_acc [B, Lq, Hq, d] and dk_acc / dv_acc
+ * [B, Lk, Hkv, d] float32, read and written (start them at zero).  All
+ * device pointers owned by the caller; tensors 16-byte aligned.  A stream-
+ * ordered workspace of 2 * B * Hq * ceil(Lq / 128) * 128 floats is
+ * allocated and freed on `stream`.  Returns RA_OK, RA_ERR_INVALID_ARG,
+ * RA_ERR_UNSUPPORTED, RA_ERR_CUDA or RA_ERR_OOM.
+ */
+int ring_attn_bwd_block_step(const void* q_chunk, const void* k_chunk, const void* v_chunk,
+                             const void* out_chunk, const void* dout_chunk, const float* lse_chunk,
+                             int64_t q_off, int64_t k_off, float* dq_acc, float* dk_acc, float* dv_acc,
+                             int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d,
+                             int causal, float scale, void* stream);
+
+/*
  * ring_attn_fwd_noalloc -- ring_attn_fwd for incremental queries
  * (cache_idx >= 0) that allocates no device memory.  The pages have no
  * counterpart; this exists for callers that cannot let a library allocate:

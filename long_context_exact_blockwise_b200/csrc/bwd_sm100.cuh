@@ -57,6 +57,7 @@ struct BwdParams {
   long long N_q, N_kv, Npad;
   long long q_pos0, k_pos0;  // global positions of q row 0 and k row 0
   int causal;
+  int accumulate;  // 0: write dq, dk, dv as bf16; 1: add into float32 dq, dk, dv
   float scale;
   float scale_log2;
   int n_qt, n_kt;  // query / key tiles
@@ -130,8 +131,8 @@ struct DkdvLayout {
   static constexpr int kV = kK + kTile;
   static constexpr int kStage0 = kV + kTile;                 // per stage: Q, dout, lse2[128], D[128]
   static constexpr int kStageBytes = 2 * kTile + 2 * kBT * 4;
-  static constexpr int kBars = kStage0 + 2 * kStageBytes;    // kv_full, qf[2], qe[2], s, p, done, drain
-  static constexpr int kMisc = kBars + 10 * 8;
+  static constexpr int kBars = kStage0 + 2 * kStageBytes;  // kv_full, qf[2], qe[2], s, p, done, drain, dp, ds
+  static constexpr int kMisc = kBars + 12 * 8;
   static constexpr int kBytes = kMisc + 16;
   // More than half the SM's shared memory: one CTA per SM, so the 512-column
   // TMEM allocation never waits on another CTA.
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
   auto BAR_QF = [&](int s) { return bar0 + 8u * (1 + s); };
   auto BAR_QE = [&](int s) { return bar0 + 8u * (3 + s); };
   const uint32_t BAR_S = bar0 + 8u * 5, BAR_P = bar0 + 8u * 6, BAR_DONE = bar0 + 8u * 7, BAR_DRAIN = bar0 + 8u * 8;
+  const uint32_t BAR_DP = bar0 + 8u * 9, BAR_DS = bar0 + 8u * 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   auto stage_q = [&](int s) { return sbase + L::kStage0 + s * L::kStageBytes; };
@@ -159,9 +161,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
   auto stage_d = [&](int s) { return stage_lse(s) + kBT; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int jt = (int)(blockIdx.x % p.n_kt);
-  const int hk = (int)((blockIdx.x / p.n_kt) % p.Hkv);
-  const int b = (int)(blockIdx.x / ((long long)p.n_kt * p.Hkv));
+  // Key-tile-major order: under a causal mask the work of a key tile falls
+  // with its index, so the longest CTAs start first and the short ones fill
+  // the tail.  The (batch, head) pairs of one key tile run side by side.
+  const int jt = (int)(blockIdx.x / ((unsigned)p.Hkv * p.B));
+  const int hk = (int)(blockIdx.x % p.Hkv);
+  const int b = (int)((blockIdx.x / p.Hkv) % p.B);
   const int j0 = jt * kBT;
   // First query tile with a query that sees key j0 (causal), else 0.
   int it0 = 0;
@@ -182,6 +187,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     mbar_init(BAR_P, 4);
     mbar_init(BAR_DONE, 1);
     mbar_init(BAR_DRAIN, 1);
+    mbar_init(BAR_DP, 1);
+    mbar_init(BAR_DS, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -229,22 +236,44 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Software pipeline over iterations w (one query tile of one head):
+      //   dV_w += P^T_w dout_w  |  S^T_{w+1}  |  dK_w += dS^T_w Q_w  |  dP^T_{w+1}
+      // so the tensor pipe works on the next tile's S^T while the
+      // elementwise warps form dS^T_w, and on dK_w / dP^T_{w+1} while they
+      // form P^T_{w+1}.  S^T_{w+1} overwrites the columns dV_w reads P^T_w
+      // from, and dP^T_{w+1} those dK_w reads dS^T_w from: tcgen05 MMAs of
+      // one thread run in issue order.  Each S / dP commit comes after the
+      // elementwise warps have passed the previous wait on the same barrier,
+      // so no barrier runs two phases ahead of its waiters.
       bool ok = mbar_wait(BAR_KV, 0, abort_flag);
       tc_fence_after();
+      if (ok && n_work > 0 && (ok = mbar_wait(BAR_QF(0), 0, abort_flag))) {
+        tc_fence_after();
+        mma_rows_x_rows<D>(T_ST, sbase + L::kK, stage_q(0));    // S^T = K Q^T
+        tc_commit(BAR_S);
+        mma_rows_x_rows<D>(T_DPT, sbase + L::kV, stage_do(0));  // dP^T = V dout^T
+        tc_commit(BAR_DP);
+      }
       for (int w = 0; w < n_work && ok; ++w) {
         const int s = w & 1;
-        if (!(ok = mbar_wait(BAR_QF(s), (w >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        // S^T = K Q^T and dP^T = V dout^T (after the previous iteration's
-        // dV / dK MMAs, which read P^T / dS^T from these columns: in order).
-        mma_rows_x_rows<D>(T_ST, sbase + L::kK, stage_q(s));
-        mma_rows_x_rows<D>(T_DPT, sbase + L::kV, stage_do(s));
-        tc_commit(BAR_S);
+        const bool more = w + 1 < n_work;
         if (!(ok = mbar_wait(BAR_P, w & 1, abort_flag))) break;
         tc_fence_after();
         mma_tmem_x_tile<D>(T_DV, T_ST, stage_do(s), w > 0);   // dV += P^T dout
+        if (more) {
+          if (!(ok = mbar_wait(BAR_QF(s ^ 1), ((w + 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          mma_rows_x_rows<D>(T_ST, sbase + L::kK, stage_q(s ^ 1));
+          tc_commit(BAR_S);
+        }
+        if (!(ok = mbar_wait(BAR_DS, w & 1, abort_flag))) break;
+        tc_fence_after();
         mma_tmem_x_tile<D>(T_DK, T_DPT, stage_q(s), w > 0);   // dK += dS^T Q
         tc_commit(BAR_QE(s));
+        if (more) {
+          mma_rows_x_rows<D>(T_DPT, sbase + L::kV, stage_do(s ^ 1));
+          tc_commit(BAR_DP);
+        }
       }
       tc_commit(BAR_DONE);
       tc_commit(BAR_DRAIN);
@@ -273,13 +302,14 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
       // q_pos0 + qt*128 + c >= k_pos0 + key, i.e. c >= cmin.
       long long cm = p.causal ? (key + p.k_pos0 - p.q_pos0) - (long long)qt * kBT : -1;
       const int cmin = (int)(cm < 0 ? 0 : (cm > kBT ? kBT : cm));
+      // Phase 1: P^T (kept in registers for phase 2), bf16 over S^T.
+      float pv[kBT];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float st[32], dpt[32];
+        float st[32];
         tmem_ld32(T_ST + lb + c * 32, st);
-        tmem_ld32(T_DPT + lb + c * 32, dpt);
         tc_wait_ld();
-        uint32_t up[16], uds[16];
+        uint32_t up[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const int q0 = c * 32 + i;
@@ -287,19 +317,37 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
           float p1 = ex2(fmaf(st[i + 1], sl, -lse2[q0 + 1]));
           if (q0 < cmin) p0 = 0.f;
           if (q0 + 1 < cmin) p1 = 0.f;
-          const float d0 = p0 * (dpt[i] - dD[q0]);
-          const float d1 = p1 * (dpt[i + 1] - dD[q0 + 1]);
+          pv[q0] = p0;
+          pv[q0 + 1] = p1;
           up[i / 2] = pack_bf16x2(p0, p1);
-          uds[i / 2] = pack_bf16x2(d0, d1);
         }
         tmem_st16(T_ST + lb + c * 16, up);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_P);
+      // Phase 2: dS^T = P^T (dP^T - D), bf16 over dP^T.
+      if (!(ok = mbar_wait(BAR_DP, w & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float dpt[32];
+        tmem_ld32(T_DPT + lb + c * 32, dpt);
+        tc_wait_ld();
+        uint32_t uds[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int q0 = c * 32 + i;
+          uds[i / 2] = pack_bf16x2(pv[q0] * (dpt[i] - dD[q0]), pv[q0 + 1] * (dpt[i + 1] - dD[q0 + 1]));
+        }
         tmem_st16(T_DPT + lb + c * 16, uds);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(BAR_P);
+        mbar_arrive(BAR_DS);
         mbar_arrive(BAR_QE(s));  // this warp is done with the stage's lse / D
       }
     }
@@ -308,34 +356,61 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
       tc_fence_after();
       const bool valid = key < p.N_kv;
       const long long off = (((long long)b * p.N_kv + (valid ? key : 0)) * p.Hkv + hk) * D;
-      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
-      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
+      if (p.accumulate) {
+        // dv += P^T dout, dk += scale dS^T Q into the caller's float32 rows
+        // (a key no query of this call sees is left as it was).
+        float* dv = static_cast<float*>(p.dv) + off;
+        float* dk = static_cast<float*>(p.dk) + off;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float a[32], g[32];
-        tmem_ld32(T_DV + lb + c * 32, a);
-        tmem_ld32(T_DK + lb + c * 32, g);
-        tc_wait_ld();
-        if (!valid) continue;
-        // A key no query sees gets a zero gradient (TMEM was never written).
+        for (int c = 0; c < D / 32; ++c) {
+          float a[32], g[32];
+          tmem_ld32(T_DV + lb + c * 32, a);
+          tmem_ld32(T_DK + lb + c * 32, g);
+          tc_wait_ld();
+          if (!valid || n_work == 0) continue;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          a[i] = n_work > 0 ? a[i] : 0.f;
-          g[i] = n_work > 0 ? g[i] * p.scale : 0.f;
+          for (int i = 0; i < 32; i += 4) {
+            float4 ov = *reinterpret_cast<float4*>(dv + c * 32 + i);
+            float4 ok4 = *reinterpret_cast<float4*>(dk + c * 32 + i);
+            ov.x += a[i]; ov.y += a[i + 1]; ov.z += a[i + 2]; ov.w += a[i + 3];
+            ok4.x = fmaf(g[i], p.scale, ok4.x);
+            ok4.y = fmaf(g[i + 1], p.scale, ok4.y);
+            ok4.z = fmaf(g[i + 2], p.scale, ok4.z);
+            ok4.w = fmaf(g[i + 3], p.scale, ok4.w);
+            *reinterpret_cast<float4*>(dv + c * 32 + i) = ov;
+            *reinterpret_cast<float4*>(dk + c * 32 + i) = ok4;
+          }
         }
+      } else {
+        __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
+        __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 wv, wk;
-          wv.x = pack_bf16x2(a[i], a[i + 1]);
-          wv.y = pack_bf16x2(a[i + 2], a[i + 3]);
-          wv.z = pack_bf16x2(a[i + 4], a[i + 5]);
-          wv.w = pack_bf16x2(a[i + 6], a[i + 7]);
-          wk.x = pack_bf16x2(g[i], g[i + 1]);
-          wk.y = pack_bf16x2(g[i + 2], g[i + 3]);
-          wk.z = pack_bf16x2(g[i + 4], g[i + 5]);
-          wk.w = pack_bf16x2(g[i + 6], g[i + 7]);
-          *reinterpret_cast<uint4*>(dv + c * 32 + i) = wv;
-          *reinterpret_cast<uint4*>(dk + c * 32 + i) = wk;
+        for (int c = 0; c < D / 32; ++c) {
+          float a[32], g[32];
+          tmem_ld32(T_DV + lb + c * 32, a);
+          tmem_ld32(T_DK + lb + c * 32, g);
+          tc_wait_ld();
+          if (!valid) continue;
+          // A key no query sees gets a zero gradient (TMEM was never written).
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            a[i] = n_work > 0 ? a[i] : 0.f;
+            g[i] = n_work > 0 ? g[i] * p.scale : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 wv, wk;
+            wv.x = pack_bf16x2(a[i], a[i + 1]);
+            wv.y = pack_bf16x2(a[i + 2], a[i + 3]);
+            wv.z = pack_bf16x2(a[i + 4], a[i + 5]);
+            wv.w = pack_bf16x2(a[i + 6], a[i + 7]);
+            wk.x = pack_bf16x2(g[i], g[i + 1]);
+            wk.y = pack_bf16x2(g[i + 2], g[i + 3]);
+            wk.z = pack_bf16x2(g[i + 4], g[i + 5]);
+            wk.w = pack_bf16x2(g[i + 6], g[i + 7]);
+            *reinterpret_cast<uint4*>(dv + c * 32 + i) = wv;
+            *reinterpret_cast<uint4*>(dk + c * 32 + i) = wk;
+          }
         }
       }
     }
@@ -354,8 +429,8 @@ struct DqLayout {
   static constexpr int kDo = kQ + kTile;
   static constexpr int kStage0 = kDo + kTile;  // per stage: K, V
   static constexpr int kStageBytes = 2 * kTile;
-  static constexpr int kBars = kStage0 + 2 * kStageBytes;  // q_full, kf[2], ke[2], s, p, done, drain
-  static constexpr int kMisc = kBars + 10 * 8;
+  static constexpr int kBars = kStage0 + 2 * kStageBytes;  // q_full, kf[2], ke[2], s[2], ds, done, drain, dp
+  static constexpr int kMisc = kBars + 12 * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024 < 120 * 1024 ? 120 * 1024 : kBytes + 1024;
 };
@@ -370,16 +445,20 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
   const uint32_t BAR_Q = bar0;
   auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
   auto BAR_KE = [&](int s) { return bar0 + 8u * (3 + s); };
-  const uint32_t BAR_S = bar0 + 8u * 5, BAR_P = bar0 + 8u * 6, BAR_DONE = bar0 + 8u * 7, BAR_DRAIN = bar0 + 8u * 8;
+  auto BAR_S = [&](int s) { return bar0 + 8u * (5 + s); };
+  const uint32_t BAR_DS = bar0 + 8u * 7, BAR_DONE = bar0 + 8u * 8, BAR_DRAIN = bar0 + 8u * 9, BAR_DP = bar0 + 8u * 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   auto stage_k = [&](int s) { return sbase + L::kStage0 + s * L::kStageBytes; };
   auto stage_v = [&](int s) { return stage_k(s) + L::kTile; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = (int)(blockIdx.x % p.n_qt);
-  const int h = (int)((blockIdx.x / p.n_qt) % p.Hq);
-  const int b = (int)(blockIdx.x / ((long long)p.n_qt * p.Hq));
+  // Query tiles from the last: under a causal mask a query tile's work grows
+  // with its index, so the longest CTAs start first.  The query heads of one
+  // KV group are adjacent and read the same K / V tiles.
+  const int qt = p.n_qt - 1 - (int)(blockIdx.x / ((unsigned)p.Hq * p.B));
+  const int h = (int)(blockIdx.x % p.Hq);
+  const int b = (int)((blockIdx.x / p.Hq) % p.B);
   const int hk = h / p.G;
   const int t0 = qt * kBT;
   // Key tiles with a key some query of this tile sees.
@@ -395,11 +474,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR_KF(s), 1);
       mbar_init(BAR_KE(s), 1);
+      mbar_init(BAR_S(s), 1);
     }
-    mbar_init(BAR_S, 1);
-    mbar_init(BAR_P, 4);
+    mbar_init(BAR_DS, 4);
     mbar_init(BAR_DONE, 1);
     mbar_init(BAR_DRAIN, 1);
+    mbar_init(BAR_DP, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -411,8 +491,9 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D)
-  const uint32_t T_S = tmem, T_DP = tmem + 128, T_DQ = tmem + 256;
+  // TMEM columns: S (two buffers) [0,128) and [128,256), dP [256,384), dQ [384, 384+D)
+  auto T_S = [&](int s) { return tmem + 128u * s; };
+  const uint32_t T_DP = tmem + 256, T_DQ = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -436,19 +517,40 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Software pipeline over key tiles j, S double-buffered in TMEM:
+      //   S_{j+1}  |  dQ += dS_j K_j  |  dP_{j+1}
+      // so S_{j+1} (and the elementwise warps' exponentials for it) overlap
+      // dS_j.  S_{j+1} goes to the buffer dQ_{j-1} read dS_{j-1} from, and
+      // dP_{j+1} over dP_j, which the warps finished with at dS_j: tcgen05
+      // MMAs of one thread run in issue order.  Each S buffer has its own
+      // barrier, and S_{j+2} is committed only after dS_j, so neither runs
+      // two phases ahead of the elementwise warps.
       bool ok = mbar_wait(BAR_Q, 0, abort_flag);
       tc_fence_after();
+      if (ok && n_jt > 0 && (ok = mbar_wait(BAR_KF(0), 0, abort_flag))) {
+        tc_fence_after();
+        mma_rows_x_rows<D>(T_S(0), sbase + L::kQ, stage_k(0));   // S = Q K^T
+        tc_commit(BAR_S(0));
+        mma_rows_x_rows<D>(T_DP, sbase + L::kDo, stage_v(0));    // dP = dout V^T
+        tc_commit(BAR_DP);
+      }
       for (int j = 0; j < n_jt && ok; ++j) {
         const int s = j & 1;
-        if (!(ok = mbar_wait(BAR_KF(s), (j >> 1) & 1, abort_flag))) break;
+        const bool more = j + 1 < n_jt;
+        if (more) {
+          if (!(ok = mbar_wait(BAR_KF(s ^ 1), ((j + 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          mma_rows_x_rows<D>(T_S(s ^ 1), sbase + L::kQ, stage_k(s ^ 1));
+          tc_commit(BAR_S(s ^ 1));
+        }
+        if (!(ok = mbar_wait(BAR_DS, j & 1, abort_flag))) break;
         tc_fence_after();
-        mma_rows_x_rows<D>(T_S, sbase + L::kQ, stage_k(s));    // S = Q K^T
-        mma_rows_x_rows<D>(T_DP, sbase + L::kDo, stage_v(s));  // dP = dout V^T
-        tc_commit(BAR_S);
-        if (!(ok = mbar_wait(BAR_P, j & 1, abort_flag))) break;
-        tc_fence_after();
-        mma_tmem_x_tile<D>(T_DQ, T_S, stage_k(s), j > 0);      // dQ += dS K
+        mma_tmem_x_tile<D>(T_DQ, T_S(s), stage_k(s), j > 0);    // dQ += dS K
         tc_commit(BAR_KE(s));
+        if (more) {
+          mma_rows_x_rows<D>(T_DP, sbase + L::kDo, stage_v(s ^ 1));
+          tc_commit(BAR_DP);
+        }
       }
       tc_commit(BAR_DONE);
       tc_commit(BAR_DRAIN);
@@ -469,54 +571,88 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     const long long klast_abs = p.causal ? t + (p.q_pos0 - p.k_pos0) : p.N_kv - 1;
     bool ok = true;
     for (int j = 0; j < n_jt; ++j) {
-      if (!(ok = mbar_wait(BAR_S, j & 1, abort_flag))) break;
+      const int s = j & 1;
+      if (!(ok = mbar_wait(BAR_S(s), (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
       const long long kl = min(klast_abs, p.N_kv - 1) - (long long)j * kBT;
       const int klast = (int)(kl < -1 ? -1 : (kl > kBT ? kBT : kl));
+      // P first (while dP may still be in the tensor pipe), then dS over S.
+      float pv[kBT];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float sv[32], dp[32];
-        tmem_ld32(T_S + lb + c * 32, sv);
+        float sv[32];
+        tmem_ld32(T_S(s) + lb + c * 32, sv);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float pe = ex2(fmaf(sv[i], sl, -lse2));
+          pv[c * 32 + i] = c * 32 + i > klast ? 0.f : pe;
+        }
+      }
+      if (!(ok = mbar_wait(BAR_DP, j & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float dp[32];
         tmem_ld32(T_DP + lb + c * 32, dp);
         tc_wait_ld();
         uint32_t uds[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const int k0 = c * 32 + i;
-          float p0 = ex2(fmaf(sv[i], sl, -lse2));
-          float p1 = ex2(fmaf(sv[i + 1], sl, -lse2));
-          if (k0 > klast) p0 = 0.f;
-          if (k0 + 1 > klast) p1 = 0.f;
-          uds[i / 2] = pack_bf16x2(p0 * (dp[i] - Dt), p1 * (dp[i + 1] - Dt));
+          uds[i / 2] = pack_bf16x2(pv[k0] * (dp[i] - Dt), pv[k0 + 1] * (dp[i + 1] - Dt));
         }
-        tmem_st16(T_S + lb + c * 16, uds);
+        tmem_st16(T_S(s) + lb + c * 16, uds);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR_P);
+      if (lane == 0) mbar_arrive(BAR_DS);
     }
     if (ok) ok = mbar_wait(BAR_DONE, 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + (((long long)b * p.N_q + (valid ? t : 0)) * p.Hq + h) * D;
+      const long long off = (((long long)b * p.N_q + (valid ? t : 0)) * p.Hq + h) * D;
+      if (p.accumulate) {
+        // dq += scale dS K into the caller's float32 row (unchanged when no
+        // key of this call is visible to the tile).
+        float* dq = static_cast<float*>(p.dq) + off;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float a[32];
-        tmem_ld32(T_DQ + lb + c * 32, a);
-        tc_wait_ld();
-        if (!valid) continue;
-        // A query that sees no key gets a zero gradient (TMEM never written).
+        for (int c = 0; c < D / 32; ++c) {
+          float a[32];
+          tmem_ld32(T_DQ + lb + c * 32, a);
+          tc_wait_ld();
+          if (!valid || n_jt == 0) continue;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) a[i] = n_jt > 0 ? a[i] * p.scale : 0.f;
+          for (int i = 0; i < 32; i += 4) {
+            float4 o = *reinterpret_cast<float4*>(dq + c * 32 + i);
+            o.x = fmaf(a[i], p.scale, o.x);
+            o.y = fmaf(a[i + 1], p.scale, o.y);
+            o.z = fmaf(a[i + 2], p.scale, o.z);
+            o.w = fmaf(a[i + 3], p.scale, o.w);
+            *reinterpret_cast<float4*>(dq + c * 32 + i) = o;
+          }
+        }
+      } else {
+        __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + off;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 w;
-          w.x = pack_bf16x2(a[i], a[i + 1]);
-          w.y = pack_bf16x2(a[i + 2], a[i + 3]);
-          w.z = pack_bf16x2(a[i + 4], a[i + 5]);
-          w.w = pack_bf16x2(a[i + 6], a[i + 7]);
-          *reinterpret_cast<uint4*>(dq + c * 32 + i) = w;
+        for (int c = 0; c < D / 32; ++c) {
+          float a[32];
+          tmem_ld32(T_DQ + lb + c * 32, a);
+          tc_wait_ld();
+          if (!valid) continue;
+          // A query that sees no key gets a zero gradient (TMEM never written).
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = n_jt > 0 ? a[i] * p.scale : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(a[i], a[i + 1]);
+            w.y = pack_bf16x2(a[i + 2], a[i + 3]);
+            w.z = pack_bf16x2(a[i + 4], a[i + 5]);
+            w.w = pack_bf16x2(a[i + 6], a[i + 7]);
+            *reinterpret_cast<uint4*>(dq + c * 32 + i) = w;
+          }
         }
       }
     }
@@ -579,8 +715,9 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
   prm.N_kv = a.N_kv;
   prm.Npad = a.Npad;
   prm.q_pos0 = a.q_pos0;
-  prm.k_pos0 = 0;
+  prm.k_pos0 = a.k_pos0;
   prm.causal = a.causal;
+  prm.accumulate = a.accumulate;
   prm.scale = a.scale;
   prm.scale_log2 = a.scale * kLog2e;
   prm.n_qt = (int)((a.N_q + kBT - 1) / kBT);

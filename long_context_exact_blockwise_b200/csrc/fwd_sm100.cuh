@@ -26,6 +26,12 @@
 //                that straddle the causal diagonal or a chunk edge), runs the
 //                exp2 online softmax, writes P (bf16) back over S, rescales O
 //                in TMEM when the row max grew, and writes the epilogue.
+//   warps 8..11  (FP8 KV cache only, single-tile CTAs) converters: the
+//                producer's TMA brings raw E4M3 tiles into their own ring of
+//                NSLOT8 slots; these warps decode each tile to bf16 in the
+//                128-byte-swizzled layout the MMAs read and publish it in the
+//                bf16 ring.  k_scale folds into the exponent scale, v_scale
+//                into the epilogue.
 // TMEM columns: S_t at [128 t, 128 t + 128) (P_t aliases its first 64
 // columns), O_t at [128 NQT + D t, ... + D).
 //
@@ -39,6 +45,8 @@
 
 #include <cstdlib>
 #include <cstring>
+
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -67,6 +75,13 @@ constexpr int kLaunchRegs = 168;
 constexpr int kRegsControl = 88;   // warps 0-3: TMA, MMA issue, TMEM allocation
 constexpr int kRegsSoftmax = 208;  // warps 4-11: the two softmax warpgroups
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * kLaunchRegs, "register split exceeds the launch");
+// Register split of the FP8-KV kernel (one query tile + a converter
+// warpgroup: 384 threads at 168 registers).
+constexpr int kRegsControl8 = 80;   // warps 0-3
+constexpr int kRegsSoftmax8 = 248;  // warps 4-7
+constexpr int kRegsConvert8 = 80;   // warps 8-11
+static_assert(128 * (kRegsControl8 + kRegsSoftmax8 + kRegsConvert8) <= 384 * kLaunchRegs,
+              "register split exceeds the launch");
 constexpr int kTileN = 128;  // keys per KV tile
 
 struct Sm100Params {
@@ -96,6 +111,8 @@ struct Sm100Params {
   int skip_loads;  // failure-detection test: the producer issues no copies, so the
                    // consumers' bounded waits expire and the kernel unwinds
   int tpt;     // tokens per tile: 128 / gpack
+  const float* k_scale;  // FP8 KV cache: [B, Hkv] dequantisation scales
+  const float* v_scale;
 };
 
 // The sequence of KV tiles one CTA visits: chunks in ring order from `home`,
@@ -161,15 +178,17 @@ __device__ __forceinline__ int clamp_key(long long x) {
   return (int)(x < kKeyClampLo ? kKeyClampLo : (x > kKeyClampHi ? kKeyClampHi : x));
 }
 
-template <int D, int NQT, int NSLOT>
+template <int D, int NQT, int NSLOT, int NSLOT8 = 0>
 struct Layout {
   static constexpr int kTileBytes = kTileM * D * 2;  // one bf16 tile of 128 rows x D
+  static constexpr int kF8Bytes = kTileN * D;        // one FP8 tile of 128 keys x D
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kQOff + NQT * kTileBytes;
-  static constexpr int kBarOff = kKVOff + NSLOT * kTileBytes;
+  static constexpr int kF8Off = kKVOff + NSLOT * kTileBytes;
+  static constexpr int kBarOff = kF8Off + NSLOT8 * kF8Bytes;
   // barriers: q, kv_full[NSLOT], kv_empty[NSLOT], s[NQT], s_consumed[NQT],
-  // p_lo[NQT], p_hi[NQT], o[NQT], drain
-  static constexpr int kNumBars = 1 + 2 * NSLOT + 5 * NQT + 1;
+  // p_lo[NQT], p_hi[NQT], o[NQT], drain, f8_full[NSLOT8], f8_empty[NSLOT8]
+  static constexpr int kNumBars = 1 + 2 * NSLOT + 5 * NQT + 1 + 2 * NSLOT8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr uint32_t kTmemCols = (NQT * (128 + D) <= 256) ? 256 : 512;
@@ -274,9 +293,52 @@ __device__ __forceinline__ void warp_arrive_after_tc(uint32_t bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
-template <int D, int NQT, int NSLOT, int MODE>
-__global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __grid_constant__ Sm100Params p) {
-  using L = Layout<D, NQT, NSLOT>;
+// Four E4M3 codes (bytes of w, lowest address first) to two bf16x2 words.
+// Every E4M3 value, subnormals included, is exact in f16 and in bf16.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const float2 f01 = __half22float2(__half2(h01));
+  const float2 f23 = __half22float2(__half2(h23));
+  lo = pack_bf16x2(f01.x, f01.y);
+  hi = pack_bf16x2(f23.x, f23.y);
+}
+
+// Decode one FP8 tile (128 keys x D codes, row-major, as the TMA copy left it)
+// into a bf16 tile in the layout a TMA copy with 128-byte swizzle produces:
+// 64-element column blocks of 128 rows x 128 bytes, the 16-byte chunk j of
+// row r stored at chunk j ^ (r mod 8).  Thread ct of the converter warpgroup
+// takes every 128th 16-code chunk; a warp reads 512 contiguous bytes.
+template <int D>
+__device__ __forceinline__ void convert_fp8_tile(const uint8_t* src, uint32_t dst, int ct) {
+  constexpr int kChunksPerRow = D / 16;
+#pragma unroll
+  for (int i = 0; i < kTileN * kChunksPerRow / 128; ++i) {
+    const int c = ct + 128 * i;
+    const int r = c / kChunksPerRow, cc = c % kChunksPerRow;
+    const uint4 w = *reinterpret_cast<const uint4*>(src + r * D + cc * 16);
+    uint32_t o[8];
+    e4m3x4_to_bf16x4(w.x, o[0], o[1]);
+    e4m3x4_to_bf16x4(w.y, o[2], o[3]);
+    e4m3x4_to_bf16x4(w.z, o[4], o[5]);
+    e4m3x4_to_bf16x4(w.w, o[6], o[7]);
+    const int j0 = (cc % 4) * 2;  // 16 codes = 32 bytes of bf16: chunks j0, j0 + 1
+    const uint32_t row = dst + (cc / 4) * (kTileN * 128) + r * 128;
+    const uint32_t a0 = row + ((uint32_t)(j0 ^ (r & 7)) << 4);
+    const uint32_t a1 = row + ((uint32_t)((j0 + 1) ^ (r & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a0), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                 : "memory");
+  }
+}
+
+template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0>
+__global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
+    fwd_sm100_kernel(const __grid_constant__ Sm100Params p) {
+  using L = Layout<D, NQT, NSLOT, NSLOT8>;
+  constexpr bool kKV8 = NSLOT8 > 0;
+  static_assert(!kKV8 || NQT == 1, "the FP8-KV kernel has one query tile");
   constexpr int kHalves = D / 64;  // 64-element (128-byte) swizzle columns per tile
   // Single-tile CTAs (short or packed queries) have no second tile to keep
   // the tensor pipe busy during a softmax, so they overlap inside the tile:
@@ -300,6 +362,8 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   auto BAR_PB = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 3 * NQT + t); };  // P_t keys 64..127, O ready
   auto BAR_O = [&](int t) { return bar0 + 8u * (1 + 2 * NSLOT + 4 * NQT + t); };
   const uint32_t BAR_DRAIN = bar0 + 8u * (1 + 2 * NSLOT + 5 * NQT);
+  auto BAR_F8_FULL = [&](int i) { return bar0 + 8u * (2 + 2 * NSLOT + 5 * NQT + i); };
+  auto BAR_F8_EMPTY = [&](int i) { return bar0 + 8u * (2 + 2 * NSLOT + 5 * NQT + NSLOT8 + i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -342,8 +406,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q(), 1);
     for (int i = 0; i < NSLOT; ++i) {
-      mbar_init(BAR_KV_FULL(i), 1);
+      mbar_init(BAR_KV_FULL(i), kKV8 ? 4 : 1);  // FP8: one arrival per converter warp
       mbar_init(BAR_KV_EMPTY(i), 1);
+    }
+    for (int i = 0; i < NSLOT8; ++i) {
+      mbar_init(BAR_F8_FULL(i), 1);
+      mbar_init(BAR_F8_EMPTY(i), 4);
     }
     for (int t = 0; t < NQT; ++t) {
       // One arrival per softmax warp that holds valid rows.
@@ -373,6 +441,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   // launch): 128 * 88 + 256 * 208 = 384 * 168.
   if (warp < 4) {
     if constexpr (NQT == 2) reg_dealloc<kRegsControl>();
+    if constexpr (kKV8) reg_dealloc<kRegsControl8>();
   }
   if (warp == 0) {
     // =========================== TMA producer ===========================
@@ -400,29 +469,44 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
       while (ok && cur.valid()) {
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
-          const uint32_t slot = issued % NSLOT;
-          const uint32_t use = issued / NSLOT;
-          if (!mbar_wait(BAR_KV_EMPTY(slot), (use & 1u) ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(BAR_KV_FULL(slot), L::kTileBytes);
           const CUtensorMap* map = kv == 0 ? &p.tm_k : &p.tm_v;
+          if constexpr (kKV8) {
+            // Raw E4M3 tile (no swizzle) into the FP8 ring; the converters
+            // fill the bf16 slot.
+            const uint32_t slot8 = issued % NSLOT8;
+            if (!mbar_wait(BAR_F8_EMPTY(slot8), ((issued / NSLOT8) & 1u) ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(BAR_F8_FULL(slot8), L::kF8Bytes);
+            tma_load_4d(sbase + L::kF8Off + slot8 * L::kF8Bytes, map, BAR_F8_FULL(slot8), 0, hk, (int)cur.k0, b);
+          } else {
+            const uint32_t slot = issued % NSLOT;
+            const uint32_t use = issued / NSLOT;
+            if (!mbar_wait(BAR_KV_EMPTY(slot), (use & 1u) ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(BAR_KV_FULL(slot), L::kTileBytes);
 #pragma unroll
-          for (int hf = 0; hf < kHalves; ++hf)
-            tma_load_4d(sbase + L::kKVOff + slot * L::kTileBytes + hf * (kTileN * 128), map, BAR_KV_FULL(slot),
-                        hf * 64, hk, (int)cur.k0, b);
+            for (int hf = 0; hf < kHalves; ++hf)
+              tma_load_4d(sbase + L::kKVOff + slot * L::kTileBytes + hf * (kTileN * 128), map, BAR_KV_FULL(slot),
+                          hf * 64, hk, (int)cur.k0, b);
+          }
           ++issued;
         }
         cur.next();
       }
       // Let the last fills land before the CTA can exit (normally already
       // consumed; this matters only when unwinding after a timeout).
-      const uint32_t first = issued > NSLOT ? issued - NSLOT : 0;
+      constexpr uint32_t kRing = kKV8 ? NSLOT8 : NSLOT;
+      const uint32_t first = issued > kRing ? issued - kRing : 0;
       for (uint32_t f = first; f < issued; ++f) {
-        const uint32_t slot = f % NSLOT;
         volatile int no_abort = 0;
-        mbar_wait(BAR_KV_FULL(slot), (f / NSLOT) & 1u, &no_abort);
+        if constexpr (kKV8)
+          mbar_wait(BAR_F8_FULL(f % NSLOT8), (f / NSLOT8) & 1u, &no_abort);
+        else
+          mbar_wait(BAR_KV_FULL(f % NSLOT), (f / NSLOT) & 1u, &no_abort);
       }
       mbar_wait(BAR_Q(), 0, abort_flag);
     }
@@ -540,9 +624,37 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
       volatile int no_abort = 0;
       mbar_wait(BAR_DRAIN, 0, &no_abort);
     }
+  } else if (kKV8 && warp >= 4 + 4 * NQT) {
+    // ============================ FP8 converters ============================
+    if constexpr (kKV8) {
+      reg_dealloc<kRegsConvert8>();
+      const int ct = (int)threadIdx.x - (128 + 128 * NQT);
+      KvCursor cur;
+      cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
+      uint32_t f = 0;  // fills converted, in the producer's order (K_j, V_j, ...)
+      bool ok = true;
+      while (ok && cur.valid()) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t slot8 = f % NSLOT8, slot = f % NSLOT;
+          if (!(ok = mbar_wait(BAR_F8_FULL(slot8), (f / NSLOT8) & 1u, abort_flag))) break;
+          if (!(ok = mbar_wait(BAR_KV_EMPTY(slot), ((f / NSLOT) & 1u) ^ 1u, abort_flag))) break;
+          convert_fp8_tile<D>(smem + L::kF8Off + slot8 * L::kF8Bytes, sbase + L::kKVOff + slot * L::kTileBytes, ct);
+          // The bf16 tile is read by the tensor cores (async proxy).
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(BAR_KV_FULL(slot));
+            mbar_arrive(BAR_F8_EMPTY(slot8));
+          }
+          ++f;
+        }
+        cur.next();
+      }
+    }
   } else if (warp >= 4) {
     // ========================= softmax warpgroups =========================
     if constexpr (NQT == 2) reg_alloc<kRegsSoftmax>();
+    if constexpr (kKV8) reg_alloc<kRegsSoftmax8>();
     const int t = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int rloc = quad * 32 + lane;  // row inside the tile == TMEM lane
@@ -558,8 +670,13 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     const bool warp_active = quad * 32 < q.nv;
     // With scale > 0 the row max is taken on raw scores and the scale is
     // folded into the exponent's FMA; otherwise scores are scaled first.
-    const bool fold = p.scale_log2 > 0.f;
-    const float sl = fold ? p.scale_log2 : 1.f;
+    // FP8 KV cache: k = code * k_scale folds into the score scale, v = code *
+    // v_scale into the final normalisation.
+    const float k_mul = kKV8 ? p.k_scale[b * p.Hkv + hk] : 1.f;
+    const float v_mul = kKV8 ? p.v_scale[b * p.Hkv + hk] : 1.f;
+    const float scale_l2 = p.scale_log2 * k_mul;
+    const bool fold = scale_l2 > 0.f;
+    const float sl = fold ? scale_l2 : 1.f;
 
     // m2: the base of the exponentials (log2 units); it trails the true row
     // max by at most kRescaleSlack, so exp2(x - m2) <= 2^kRescaleSlack and O
@@ -609,7 +726,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
         if constexpr (kSplitS) warp_arrive_after_tc(BAR_SC(t), lane);
         if (!fold) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] *= p.scale_log2;
+          for (int c = 0; c < 128; ++c) s[c] *= scale_l2;
         }
         const bool masked = tile_needs_mask(q, cur.k0, cur.kend, p.causal);
         if (masked) {
@@ -718,7 +835,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
     if (ok && warp_active) {
       tc_fence_after();
       if (MODE == kModeFinal || MODE == kModeSplit) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = l > 0.f ? v_mul / l : 0.f;
         const long long ooff =
             (((long long)(MODE == kModeSplit ? sigma * p.B + b : b) * p.N_q + row) * p.Hq + head) * D;
 #pragma unroll
@@ -786,12 +903,13 @@ __global__ void __launch_bounds__(128 + 128 * NQT, 1) fwd_sm100_kernel(const __g
   if (warp == 2) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-template <int D, int NQT, int NSLOT, int MODE>
+template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0>
 cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) {
-  using L = Layout<D, NQT, NSLOT>;
-  auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE>;
+  using L = Layout<D, NQT, NSLOT, NSLOT8>;
+  auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE, NSLOT8>;
   static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
-  if constexpr (NQT == 2) {
+  constexpr int kThreads = 128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0);
+  if constexpr (NQT == 2 || NSLOT8 > 0) {
     // The in-kernel register split assumes exactly kLaunchRegs per thread.
     static int regs = -1;
     if (regs < 0) {
@@ -813,8 +931,22 @@ cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) 
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
   }
-  kern<<<(unsigned)grid, 128 + 128 * NQT, L::kAlloc, st>>>(prm);
+  kern<<<(unsigned)grid, kThreads, L::kAlloc, st>>>(prm);
   return count_launch(cudaGetLastError());
+}
+
+// FP8 codes, one row of d bytes per (token, head): 128-key boxes without
+// swizzle (the converters re-lay them out).
+CUresult encode_map_u8(CUtensorMap* m, const void* base, int d, int H, long long N, int B) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return CUDA_ERROR_NOT_FOUND;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)H * d, (cuuint64_t)N * H * d};
+  cuuint32_t box[4] = {(cuuint32_t)d, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N, int B, int box_heads = 1) {
@@ -841,7 +973,9 @@ Sm100Geometry sm100_geometry(const ProblemArgs& a, int mode) {
   g.gshift = 0;
   while ((1 << g.gshift) < g.gpack) ++g.gshift;
   g.tpt = kTileM / g.gpack;
-  g.two = a.N_q * g.gpack > kTileM;  // two query tiles per CTA share each K/V tile
+  // Two query tiles per CTA share each K/V tile (not with an FP8 cache,
+  // whose CTAs carry a converter warpgroup instead).
+  g.two = a.N_q * g.gpack > kTileM && !a.kv8;
   const long long tok_per_cta = (long long)(g.two ? 2 : 1) * g.tpt;
   g.n_qblk = (int)((a.N_q + tok_per_cta - 1) / tok_per_cta);
   g.ctas_per_split = (long long)g.n_qblk * a.B * a.Hkv * (pack ? 1 : G);
@@ -853,10 +987,18 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   const Sm100Geometry geo = sm100_geometry(a, mode);
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
-  if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B, geo.gpack) != CUDA_SUCCESS ||
-      encode_map(&prm.tm_k, a.k, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS ||
-      encode_map(&prm.tm_v, a.v, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS)
+  if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B, geo.gpack) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (a.kv8) {
+    if (mode == kModeState || encode_map_u8(&prm.tm_k, a.k, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS ||
+        encode_map_u8(&prm.tm_v, a.v, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    prm.k_scale = a.k_scale;
+    prm.v_scale = a.v_scale;
+  } else if (encode_map(&prm.tm_k, a.k, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS ||
+             encode_map(&prm.tm_v, a.v, a.d, a.Hkv, a.N_kv, a.B) != CUDA_SUCCESS) {
+    return cudaErrorInvalidValue;
+  }
   prm.out = a.out;
   prm.lse = a.lse;
   prm.o_part = a.o_part;
@@ -897,6 +1039,15 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
     case kModeFinal: return launch_cfg<D_, NQT_, NS_, kModeFinal>(prm, grid, st); \
     case kModeSplit: return launch_cfg<D_, NQT_, NS_, kModeSplit>(prm, grid, st); \
     default: return launch_cfg<D_, NQT_, NS_, kModeState>(prm, grid, st);        \
+  }
+  if (a.kv8) {
+    // One query tile, bf16 ring, FP8 ring (d=128: 32 + 4 x 32 + 4 x 16 = 224 KB).
+    if (a.d == 64) {
+      if (mode == kModeFinal) return launch_cfg<64, 1, 6, kModeFinal, 8>(prm, grid, st);
+      return launch_cfg<64, 1, 6, kModeSplit, 8>(prm, grid, st);
+    }
+    if (mode == kModeFinal) return launch_cfg<128, 1, 4, kModeFinal, 4>(prm, grid, st);
+    return launch_cfg<128, 1, 4, kModeSplit, 4>(prm, grid, st);
   }
   if (a.d == 64) {
     if (two) { RA_LAUNCH(64, 2, 8) } else { RA_LAUNCH(64, 1, 8) }

@@ -50,6 +50,9 @@ struct ProblemArgs {
   int P;
   int S;            // KV splits (kModeSplit), 1 otherwise
   int out_f32;      // kModeFinal: 1 = float32 out, 0 = bf16 out
+  int kv8;          // 1: k and v are FP8 E4M3 codes, dequantised by k_scale / v_scale [B, Hkv]
+  const float* k_scale;
+  const float* v_scale;
 };
 
 // Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.
@@ -92,8 +95,9 @@ struct BwdArgs {
   float* ws_d;     // [B, Hq, Npad]
   int B, Hq, Hkv, d;
   long long N_q, N_kv, Npad;
-  long long q_pos0;
+  long long q_pos0, k_pos0;  // global positions of q row 0 and k row 0
   int causal;
+  int accumulate;  // 0: dq, dk, dv are bf16 outputs; 1: float32 accumulators (+=)
   float scale;
 };
 cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t stream);

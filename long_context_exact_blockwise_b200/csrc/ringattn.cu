@@ -179,35 +179,26 @@ int ring_attn_sync_status(void* stream) {
   return status;
 }
 
-int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
-                  int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
-                  void* stream) {
-  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
-  if (r != RA_OK) return r;
-  if (B == 0 || N_q == 0) return RA_OK;
-  int num_sms = 148;
-  if ((r = check_device(&num_sms)) != RA_OK) return r;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+}  // extern "C"
 
-  ProblemArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
-  a.N_q = N_q; a.N_kv = N_kv;
-  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
-  a.k_pos0 = 0;
-  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.S = 1; a.out_f32 = 0;
+namespace {
 
-  if (cache_idx < 0) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd");
+// The bf16 tensor-core forward (and its FP8-KV variant) for validated
+// arguments: one launch for prefill, or split-KV partials merged by their
+// log-sum-exp weights for incremental queries.
+// a.S == 1: prefill, one launch; a.S == 0: incremental queries, the split
+// count is chosen here.
+int run_fwd(ProblemArgs a, int num_sms, cudaStream_t st, const char* what) {
+  if (a.S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, what);
 
   // Incremental query: split the ring steps over S CTAs per query block and
   // merge the partials by their log-sum-exp weights.
   const long long items = sm100_geometry(a, kModeSplit).ctas_per_split;
-  const int S = choose_splits(items, P, num_sms, N_q);
-  if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, "ring_attn_fwd");
+  const int S = choose_splits(items, a.P, num_sms, a.N_q);
+  if (S == 1) return finish(launch_fwd_sm100(a, kModeFinal, st), st, what);
 
-  const size_t o_bytes = (size_t)S * B * N_q * Hq * d * sizeof(float);
-  const size_t l_bytes = (size_t)S * B * Hq * N_q * sizeof(float);
+  const size_t o_bytes = (size_t)S * a.B * a.N_q * a.Hq * a.d * sizeof(float);
+  const size_t l_bytes = (size_t)S * a.B * a.Hq * a.N_q * sizeof(float);
   void* ws = nullptr;
   if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
     t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
@@ -223,10 +214,57 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
   a.o_part = static_cast<float*>(ws);
   a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
   e = launch_fwd_sm100(a, kModeSplit, st);
-  if (e == cudaSuccess) e = launch_lse_merge(a.o_part, a.lse_part, S, out, lse, B, Hq, N_q, d, 0, st);
+  if (e == cudaSuccess) e = launch_lse_merge(a.o_part, a.lse_part, S, a.out, a.lse, a.B, a.Hq, a.N_q, a.d, 0, st);
   cudaError_t ef = cudaFreeAsync(ws, st);
   if (e == cudaSuccess) e = ef;
-  return finish(e, st, "ring_attn_fwd(split)");
+  return finish(e, st, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                  int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                  void* stream) {
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N_q == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv;
+  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.k_pos0 = 0;
+  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0;
+  a.S = cache_idx < 0 ? 1 : 0;  // 0: choose a split count
+  return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd");
+}
+
+int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const float* k_scale, const float* v_scale,
+                        void* out, float* lse, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
+                        int64_t chunk, int P, int64_t cache_idx, float scale, void* stream) {
+  if (!k_scale || !v_scale) return RA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u) return RA_ERR_INVALID_ARG;
+  int r = validate_fwd(q, k8, v8, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N_q == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k8; a.v = v8; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N_q; a.N_kv = N_kv;
+  a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.k_pos0 = 0;
+  a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0;
+  a.kv8 = 1; a.k_scale = k_scale; a.v_scale = v_scale;
+  a.S = cache_idx < 0 ? 1 : 0;
+  return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd_fp8kv");
 }
 
 int ring_attn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B, int Hq,
@@ -310,19 +348,15 @@ int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, fl
                 "lse_merge");
 }
 
-int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
-                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
-                  int64_t cache_idx, float scale, void* stream) {
-  if (!dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
-  if (!(aligned16(dout) && aligned16(dq) && aligned16(dk) && aligned16(dv))) return RA_ERR_INVALID_ARG;
-  // Same shape rules as ring_attn_fwd (one chunk spanning the sequence).
-  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, N_kv, 1, cache_idx, scale, true);
-  if (r != RA_OK) return r;
-  if (B == 0 || N_q == 0) return RA_OK;
-  if ((r = check_device(nullptr)) != RA_OK) return r;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long Npad = (N_q + 127) / 128 * 128;
-  const size_t ws_bytes = (size_t)2 * B * Hq * Npad * sizeof(float);
+}  // extern "C"
+
+namespace {
+
+// Workspace (lse * log2 e and D per query row, padded to 128 rows), then the
+// three backward kernels.  Arguments are already validated.
+int run_bwd(ra::BwdArgs a, const char* what, cudaStream_t st) {
+  a.Npad = (a.N_q + 127) / 128 * 128;
+  const size_t ws_bytes = (size_t)2 * a.B * a.Hq * a.Npad * sizeof(float);
   if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
     t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
     return RA_ERR_OOM;
@@ -334,20 +368,71 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
     t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
     return RA_ERR_OOM;
   }
+  a.ws_lse2 = static_cast<float*>(ws);
+  a.ws_d = a.ws_lse2 + (size_t)a.B * a.Hq * a.Npad;
+  e = launch_bwd_sm100(a, st);
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
+  return finish(e, st, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
+                  int64_t cache_idx, float scale, void* stream) {
+  if (!dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
+  if (!(aligned16(dout) && aligned16(dq) && aligned16(dk) && aligned16(dv))) return RA_ERR_INVALID_ARG;
+  // Same shape rules as ring_attn_fwd (one chunk spanning the sequence).
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, N_kv, 1, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N_q == 0) return RA_OK;
+  if ((r = check_device(nullptr)) != RA_OK) return r;
   BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.lse = lse;
   a.dq = dq; a.dk = dk; a.dv = dv;
-  a.ws_lse2 = static_cast<float*>(ws);
-  a.ws_d = a.ws_lse2 + (size_t)B * Hq * Npad;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
-  a.N_q = N_q; a.N_kv = N_kv; a.Npad = Npad;
+  a.N_q = N_q; a.N_kv = N_kv;
   a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+  a.k_pos0 = 0;
   a.causal = causal; a.scale = scale;
-  e = launch_bwd_sm100(a, st);
-  cudaError_t ef = cudaFreeAsync(ws, st);
-  if (e == cudaSuccess) e = ef;
-  return finish(e, st, "ring_attn_bwd");
+  a.accumulate = 0;
+  return run_bwd(a, "ring_attn_bwd", static_cast<cudaStream_t>(stream));
+}
+
+int ring_attn_bwd_block_step(const void* q_chunk, const void* k_chunk, const void* v_chunk, const void* out_chunk,
+                             const void* dout_chunk, const float* lse_chunk, int64_t q_off, int64_t k_off,
+                             float* dq_acc, float* dk_acc, float* dv_acc, int B, int Hq, int Hkv, int64_t Lq,
+                             int64_t Lk, int d, int causal, float scale, void* stream) {
+  if (!q_chunk || !k_chunk || !v_chunk || !out_chunk || !dout_chunk || !lse_chunk) return RA_ERR_INVALID_ARG;
+  if (!dq_acc || !dk_acc || !dv_acc) return RA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (Lq < 0 || Lk < 0 || Lq > kMaxTokens || Lk > kMaxTokens) return RA_ERR_INVALID_ARG;
+  if (q_off < 0 || k_off < 0) return RA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (!(aligned16(q_chunk) && aligned16(k_chunk) && aligned16(v_chunk) && aligned16(out_chunk) &&
+        aligned16(dout_chunk) && aligned16(dq_acc) && aligned16(dk_acc) && aligned16(dv_acc)))
+    return RA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse_chunk) & 3u) return RA_ERR_INVALID_ARG;
+  if (B == 0 || Lq == 0 || Lk == 0) return RA_OK;
+  int r = check_device(nullptr);
+  if (r != RA_OK) return r;
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q_chunk; a.k = k_chunk; a.v = v_chunk; a.out = out_chunk; a.dout = dout_chunk; a.lse = lse_chunk;
+  a.dq = dq_acc; a.dk = dk_acc; a.dv = dv_acc;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = Lq; a.N_kv = Lk;
+  a.q_pos0 = q_off;
+  a.k_pos0 = k_off;
+  a.causal = causal; a.scale = scale;
+  a.accumulate = 1;
+  return run_bwd(a, "ring_attn_bwd_block_step", static_cast<cudaStream_t>(stream));
 }
 
 int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
-    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_bwd", "ring_attn_block_step", "ring_attn_finalize",
+    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_fwd_fp8kv", "ring_attn_bwd", "ring_attn_bwd_block_step", "ring_attn_block_step", "ring_attn_finalize",
     "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
@@ -54,7 +54,9 @@ _SIGS = {
     "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_fwd_fp8kv": [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
+    "ring_attn_bwd_block_step": [_p, _p, _p, _p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _p],
     "ring_attn_block_step": [_p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _i, _p],
     "ring_attn_finalize": [_p, _p, _p, _p, _p, _i, _i, _l, _i, _i, _p],
     "lse_merge": [_p, _p, _i, _p, _p, _i, _i, _l, _i, _i, _p],
@@ -178,6 +180,36 @@ def ring_attn_fwd_noalloc(q, k, v, *, causal: bool, P: int, cache_idx: int, chun
                 stream)
 
 
+def ring_attn_fwd_fp8kv(q, k8, v8, k_scale, v_scale, *, causal: bool, P: int, chunk: Optional[int] = None,
+                        cache_idx=None, scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """Forward over an FP8 E4M3 KV cache: q bf16 [B,N_q,Hq,d]; k8/v8 uint8 codes
+    [B,N_kv,Hkv,d]; k_scale/v_scale float32 [B,Hkv] -> (out bf16, lse f32)."""
+    _need(q, "q", torch.bfloat16)
+    for t, n in ((k8, "k8"), (v8, "v8")):
+        _need(t, n, torch.uint8)
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, n, torch.float32)
+    B, N_q, Hq, d = q.shape
+    _, N_kv, Hkv, dk = k8.shape
+    if k8.shape != v8.shape or dk != d or k8.shape[0] != B:
+        raise ValueError("k8 and v8 must be [B, N_kv, Hkv, d] matching q")
+    if tuple(k_scale.shape) != (B, Hkv) or tuple(v_scale.shape) != (B, Hkv):
+        raise ValueError("k_scale and v_scale must be [B, Hkv]")
+    if chunk is None:
+        chunk = N_kv // P if P > 0 else 0
+    ci = -1 if cache_idx is None else int(cache_idx)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    _need(out, "out", torch.bfloat16)
+    _need(lse, "lse", torch.float32)
+    st = lib.ring_attn_fwd_fp8kv(_ptr(q), _ptr(k8), _ptr(v8), _ptr(k_scale), _ptr(v_scale), _ptr(out), _ptr(lse),
+                                 B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)), int(chunk), int(P), ci, sc,
+                                 _stream(stream, q.device))
+    _check(st, "ring_attn_fwd_fp8kv")
+    return out, lse
+
+
 def ring_attn_bwd(q, k, v, out, dout, lse, *, causal: bool, cache_idx=None, scale: Optional[float] = None,
                   dq=None, dk=None, dv=None, stream=None):
     """Gradients (dq, dk, dv) of ring_attn_fwd's output for upstream dout (bf16)."""
@@ -195,6 +227,27 @@ def ring_attn_bwd(q, k, v, out, dout, lse, *, causal: bool, cache_idx=None, scal
                            _ptr(dv), B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)), ci, sc, _stream(stream, q.device))
     _check(st, "ring_attn_bwd")
     return dq, dk, dv
+
+
+def ring_attn_bwd_block_step(q_chunk, k_chunk, v_chunk, out_chunk, dout_chunk, lse_chunk, q_off: int, k_off: int,
+                             dq_acc, dk_acc, dv_acc, *, causal: bool, scale: Optional[float] = None,
+                             stream=None) -> None:
+    """Add one ring visit's share of (dq, dk, dv) into float32 accumulators, in place."""
+    for t, n in ((q_chunk, "q_chunk"), (k_chunk, "k_chunk"), (v_chunk, "v_chunk"), (out_chunk, "out_chunk"),
+                 (dout_chunk, "dout_chunk")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((lse_chunk, "lse_chunk"), (dq_acc, "dq_acc"), (dk_acc, "dk_acc"), (dv_acc, "dv_acc")):
+        _need(t, n, torch.float32)
+    B, Lq, Hq, d = q_chunk.shape
+    _, Lk, Hkv, _ = k_chunk.shape
+    if dq_acc.shape != q_chunk.shape or dk_acc.shape != k_chunk.shape or dv_acc.shape != v_chunk.shape:
+        raise ValueError("accumulator shapes must match q_chunk / k_chunk / v_chunk")
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.ring_attn_bwd_block_step(_ptr(q_chunk), _ptr(k_chunk), _ptr(v_chunk), _ptr(out_chunk),
+                                      _ptr(dout_chunk), _ptr(lse_chunk), int(q_off), int(k_off), _ptr(dq_acc),
+                                      _ptr(dk_acc), _ptr(dv_acc), B, Hq, Hkv, Lq, Lk, d, int(bool(causal)), sc,
+                                      _stream(stream, q_chunk.device))
+    _check(st, "ring_attn_bwd_block_step")
 
 
 def ring_attn(q, k, v, *, causal: bool, P: int, cache_idx=None, scale=None, stream=None):

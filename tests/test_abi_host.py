@@ -114,3 +114,38 @@ def test_block_step_finalize_merge_validation():
     assert L.lse_merge(FAKE, FAKE, 0, FAKE, FAKE, 1, 2, 8, 64, 0, None) == ra.RA_ERR_INVALID_ARG
     assert L.lse_merge(None, FAKE, 2, FAKE, FAKE, 1, 2, 8, 64, 0, None) == ra.RA_ERR_INVALID_ARG
     assert L.lse_merge(FAKE, FAKE, 2, FAKE, FAKE, 1, 2, 0, 64, 0, None) == ra.RA_OK
+
+
+def test_bwd_block_step_validation():
+    ra = _lib()
+    L = ra.lib
+    # q, k, v, out, dout, lse, q_off, k_off, dq, dk, dv, B, Hq, Hkv, Lq, Lk, d, causal, scale, stream
+    ok_args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, FAKE, FAKE, FAKE, 1, 4, 2, 128, 128, 64, 1, 0.1, None)
+    assert L.ring_attn_bwd_block_step(*ok_args) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
+    for i, val in ((6, -1), (7, -5), (12, 3), (16, 96), (17, 2), (18, float("nan"))):
+        bad = list(ok_args); bad[i] = val
+        assert L.ring_attn_bwd_block_step(*bad) == ra.RA_ERR_INVALID_ARG, i
+    for i in (0, 3, 4, 5, 8, 9, 10):
+        bad = list(ok_args); bad[i] = None
+        assert L.ring_attn_bwd_block_step(*bad) == ra.RA_ERR_INVALID_ARG, i
+    bad = list(ok_args); bad[9] = ctypes.c_void_p(0x10004)  # dk accumulator not 16-byte aligned
+    assert L.ring_attn_bwd_block_step(*bad) == ra.RA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[15] = 0  # Lk == 0: nothing to add
+    assert L.ring_attn_bwd_block_step(*bad) == ra.RA_OK
+
+
+def test_fp8kv_validation():
+    ra = _lib()
+    L = ra.lib
+    # q, k8, v8, k_scale, v_scale, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, stream
+    ok_args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 1, 256, 128, 1, 128, 2, 255, 0.1, None]
+    assert L.ring_attn_fwd_fp8kv(*ok_args) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
+    for i in (3, 4):
+        bad = list(ok_args); bad[i] = None
+        assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG, i
+    bad = list(ok_args); bad[3] = ctypes.c_void_p(0x10002)  # k_scale not 4-byte aligned
+    assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[12] = 96
+    assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[14] = 100  # N_kv != P * chunk
+    assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG

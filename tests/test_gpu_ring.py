@@ -40,3 +40,19 @@ def test_ring_driver_cuda_compute(one_rank_group, dtype, causal):
     ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
     assert np.max(np.abs(out.float().cpu().numpy() - ro)) <= TOL_OUT[dtype]
     assert np.max(np.abs(lse.cpu().numpy() - rl)) <= TOL_LSE
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_driver_cuda_backward(one_rank_group, causal):
+    from long_context_exact_blockwise_b200.ring import ring_attention, ring_attention_bwd
+    w = workloads.small(B=2, Hq=4, Hkv=2, N_q=384, d=128, causal=causal, P=1, seed=91)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    dout = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(92),
+                       device="cuda").to(torch.bfloat16)
+    out, lse = ring_attention(q, k, v, causal=causal, scale=w.scale)
+    dq, dk, dv = ring_attention_bwd(q, k, v, out, dout, lse, causal=causal, scale=w.scale)
+    torch.cuda.synchronize()
+    ref = oracle.attention_bwd_ref(q, k, v, dout, causal=causal, scale=w.scale)
+    for got, r in zip((dq, dk, dv), ref):
+        g = got.float().cpu().numpy()
+        assert np.all(np.abs(g - r) <= 2e-2 + 2e-2 * np.abs(r))

@@ -96,6 +96,67 @@ def test_ring_protocol_matches_full_attention(world, case):
         assert eo <= 1e-10 and el <= 1e-10, (r, eo, el)
 
 
+def _oracle_bwd_step():
+    import oracle
+
+    def block_step_bwd(q, k, v, out, dout, lse, q_off, k_off, dq, dk, dv, *, causal, scale):
+        delta = torch.einsum("bthe,bthe->bht", dout, out)
+        a, b, c = oracle.block_step_bwd_ref(q, k, v, dout, lse, delta, q_off, k_off, dq, dk, dv, causal=causal,
+                                            scale=scale)
+        dq.copy_(torch.from_numpy(a))
+        dk.copy_(torch.from_numpy(b))
+        dv.copy_(torch.from_numpy(c))
+
+    return block_step_bwd
+
+
+def _bwd_worker(rank, world, port, case, results):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import workloads
+        from long_context_exact_blockwise_b200.ring import ring_attention_bwd
+
+        B, Hq, Hkv, L, d, causal = case
+        w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
+                            seed=31 + world)
+        q, k, v = (x.double() for x in workloads.make_qkv(w))
+        dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5), dtype=torch.float64)
+        out, lse = (torch.from_numpy(x) for x in oracle.attention_ref(q, k, v, causal=causal, scale=w.scale))
+        sl = slice(rank * L, (rank + 1) * L)
+        chunks = [x[:, sl].contiguous() for x in (q, k, v, out, dout)]
+        before = [x.clone() for x in chunks]
+        dq, dk, dv = ring_attention_bwd(*chunks, lse[:, :, sl].contiguous(), causal=causal, scale=w.scale,
+                                        block_step_bwd=_oracle_bwd_step())
+        assert all(torch.equal(a, b) for a, b in zip(before, chunks))
+        rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=causal, scale=w.scale)
+        results[rank] = tuple(float(np.max(np.abs(g.numpy() - r[:, sl]))) for g, r in ((dq, rq), (dk, rk), (dv, rv)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("case", [(1, 2, 2, 16, 8, True), (2, 4, 2, 12, 8, False), (1, 4, 1, 9, 4, True)])
+def test_ring_backward_protocol_matches_full_gradient(world, case):
+    ctx = mp.get_context("spawn")
+    results = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, case, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0, f"rank exited with {p.exitcode}"
+    assert sorted(results.keys()) == list(range(world))
+    for r, errs in results.items():
+        assert max(errs) <= 1e-10, (r, errs)
+
+
 def test_ring_visit_order_matches_schedule_figure():
     from long_context_exact_blockwise_b200.ring import ring_visit_order
     # 4 ranks: GPU0 holds K0, K1, K2, K3 at steps 0..3; GPU1 holds K1, K2, K3, K0.
