@@ -30,6 +30,7 @@ from .attention import (
     attention_bwd_ref,
     attention_fp8kv_ref,
     attention_ref,
+    attention_window_anchor_ref,
     block_step_bwd_ref,
     block_step_ref,
     decode_e4m3,
@@ -40,12 +41,14 @@ from .attention import (
     ring_ref,
     ring_visit_chunk,
     query_home_chunk,
+    window_anchor_visible,
 )
 
 __all__ = [
     "attention_bwd_ref",
     "attention_fp8kv_ref",
     "attention_ref",
+    "attention_window_anchor_ref",
     "block_step_bwd_ref",
     "block_step_ref",
     "decode_e4m3",
@@ -56,4 +59,5 @@ __all__ = [
     "ring_ref",
     "ring_visit_chunk",
     "query_home_chunk",
+    "window_anchor_visible",
 ]

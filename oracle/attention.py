@@ -447,3 +447,57 @@ def _u8(x) -> np.ndarray:
     if hasattr(x, "detach"):
         x = x.detach().cpu().numpy()
     return np.asarray(x, dtype=np.uint8)
+
+
+def window_anchor_visible(q_pos, k_pos, n: int, window: int, anchor_period: int) -> np.ndarray:
+    """[len(q_pos), len(k_pos)] boolean: the sparse mask of "Ring Attention:
+    the secret of million-token context" §4.3 (sparse attention mask), for a
+    sequence of n tokens attending to itself.
+
+    Query i sees the local window j in [max(0, i - window), i], and the
+    anchors of its period: a = (i // anchor_period) * anchor_period, the key
+    a, the key a - 1 when a > 0, and the key a + anchor_period when
+    a < n - anchor_period (that last anchor lies after i).
+    """
+    qp = np.asarray(q_pos, dtype=np.int64)[:, None]
+    kp = np.asarray(k_pos, dtype=np.int64)[None, :]
+    vis = (kp <= qp) & (kp >= np.maximum(0, qp - window))
+    a = (qp // anchor_period) * anchor_period
+    vis |= kp == a
+    vis |= (a > 0) & (kp == a - 1)
+    vis |= (a < n - anchor_period) & (kp == a + anchor_period)
+    return vis
+
+
+def attention_window_anchor_ref(q, k, v, *, window: int, anchor_period: int, scale: float, rows=None, heads=None):
+    """Exact attention restricted to the window-and-anchor mask
+    (window_anchor_visible) of a square prefill: N_q == N_kv == n, query t at
+    position t.  Every row keeps its full (masked) score row; rows and heads
+    restrict the computation to a sample as in attention_ref.
+    Returns (out [B, R, Hh, d], lse [B, Hh, R]) as float64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape[1] != N:
+        raise ValueError("the window-and-anchor mask is defined for N_q == N_kv")
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    heads = list(range(Hq)) if heads is None else list(heads)
+    out = np.zeros((B, rows.shape[0], len(heads), d), dtype=np.float64)
+    lse = np.full((B, len(heads), rows.shape[0]), NEG_INF, dtype=np.float64)
+    k_pos = np.arange(N, dtype=np.int64)
+    for b in range(B):
+        for hi, h in enumerate(heads):
+            hk = _kv_head(h, Hq, Hkv)
+            blk = max(1, min(_ROW_BLOCK, (1 << 25) // max(1, N)))
+            for r0 in range(0, rows.shape[0], blk):
+                r = rows[r0:r0 + blk]
+                s = scale * (q[b, r, h, :] @ k[b, :, hk, :].T)
+                s = np.where(window_anchor_visible(r, k_pos, N, window, anchor_period), s, NEG_INF)
+                w, m, l = _softmax_rows(s)
+                has = l > 0
+                o = np.zeros((r.shape[0], d))
+                o[has] = (w[has] @ v[b, :, hk, :]) / l[has, None]
+                out[b, r0:r0 + r.shape[0], hi, :] = o
+                lse[b, hi, r0:r0 + r.shape[0]] = np.where(has, m + np.log(np.where(has, l, 1.0)), NEG_INF)
+    return out, lse

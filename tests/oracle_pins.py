@@ -453,6 +453,52 @@ def pin_fp8kv_attention(O):
     _close(l3, lse, 1e-12, "v_scale leaves lse")
 
 
+def _torch_window_anchor_mask(n, window, period):
+    """The window-and-anchor mask built with torch band and scatter ops."""
+    ones = torch.ones(n, n, dtype=torch.bool)
+    band = torch.tril(ones) & torch.triu(ones, diagonal=-window)   # i - window <= j <= i
+    rows = torch.arange(n)
+    a = rows - rows % period
+    m = band.clone()
+    m[rows, a] = True
+    lo = a > 0
+    m[rows[lo], a[lo] - 1] = True
+    hi = a + period < n
+    m[rows[hi], a[hi] + period] = True
+    return m
+
+
+def pin_window_anchor(O):
+    # The sparse mask against an independent torch construction, attention
+    # under it against float64 SDPA with that mask, and the reductions that
+    # must hold: window and period covering the sequence give causal
+    # attention; window 0 leaves each row its own key plus the anchors.
+    for n, W, A in [(12, 2, 4), (40, 7, 8), (33, 0, 16), (64, 100, 64), (50, 5, 10)]:
+        got = O.window_anchor_visible(np.arange(n), np.arange(n), n, W, A)
+        ref = _torch_window_anchor_mask(n, W, A).numpy()
+        assert np.array_equal(got, ref), f"window/anchor mask n={n} W={W} A={A}"
+    B, N, Hq, Hkv, d, W, A, scale = 2, 48, 4, 2, 8, 5, 16, 0.35
+    q, k, v = _rand((B, N, Hq, d), 230), _rand((B, N, Hkv, d), 231), _rand((B, N, Hkv, d), 232)
+    out, lse = O.attention_window_anchor_ref(q, k, v, window=W, anchor_period=A, scale=scale)
+    mask = _torch_window_anchor_mask(N, W, A)
+    G = Hq // Hkv
+    kr, vr = k.repeat_interleave(G, dim=2), v.repeat_interleave(G, dim=2)
+    ro = F.scaled_dot_product_attention(q.transpose(1, 2), kr.transpose(1, 2), vr.transpose(1, 2), attn_mask=mask,
+                                        scale=scale).transpose(1, 2)
+    sc = (torch.einsum("bqhd,bkhd->bhqk", q, kr) * scale).masked_fill(~mask, float("-inf"))
+    _close(out, ro.numpy(), 1e-10, "window/anchor out vs sdpa")
+    _close(lse, torch.logsumexp(sc, dim=-1).numpy(), 1e-10, "window/anchor lse vs sdpa")
+    rows = np.array([0, 5, 17, 47])
+    o_s, l_s = O.attention_window_anchor_ref(q, k, v, window=W, anchor_period=A, scale=scale, rows=rows,
+                                             heads=[3, 0])
+    _close(o_s, out[:, rows][:, :, [3, 0]], 1e-13, "window/anchor sampled rows")
+    _close(l_s, lse[:, [3, 0]][:, :, rows], 1e-13, "window/anchor sampled lse")
+    oc, lc = O.attention_window_anchor_ref(q, k, v, window=N, anchor_period=N, scale=scale)
+    rc, rlc = O.attention_ref(q, k, v, causal=True, scale=scale)
+    _close(oc, rc, 1e-12, "full window = causal")
+    _close(lc, rlc, 1e-12, "full window = causal (lse)")
+
+
 ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
             pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference,
-            pin_backward_ring, pin_fp8_decode, pin_fp8kv_attention]
+            pin_backward_ring, pin_fp8_decode, pin_fp8kv_attention, pin_window_anchor]

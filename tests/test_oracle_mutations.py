@@ -59,6 +59,12 @@ MUTATIONS = [
     ("fp8 v scaled by k_scale", "v = decode_e4m3(_u8(v8)) * vs[", "v = decode_e4m3(_u8(v8)) * ks["),
     ("fp8 scale transposed", "k = decode_e4m3(_u8(k8)) * ks[:, None, :, None]",
      "k = decode_e4m3(_u8(k8)) * ks.T[:, None, :, None]"),
+    ("window one key short", "(kp >= np.maximum(0, qp - window))", "(kp > np.maximum(0, qp - window))"),
+    ("window not causal", "vis = (kp <= qp) & (kp >= np.maximum", "vis = (kp <= qp + 1) & (kp >= np.maximum"),
+    ("anchor minus one dropped", "vis |= (a > 0) & (kp == a - 1)", "vis |= (a > 0) & (kp == a)"),
+    ("future anchor one early", "vis |= (a < n - anchor_period) & (kp == a + anchor_period)",
+     "vis |= (a < n - anchor_period) & (kp == a + anchor_period - 1)"),
+    ("anchor not floored", "a = (qp // anchor_period) * anchor_period", "a = qp // anchor_period"),
     ("bwd visit dk from dout", "dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])",
      "dk[b, :, hk, :] += scale * (ds.T @ do[b, :, h, :])"),
 ]
