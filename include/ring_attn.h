@@ -179,7 +179,8 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
  * them (q, out bf16; lse float32; same shapes, causal, chunk, P, cache_idx
  * and scale rules; incremental queries use split-KV partials and a stream-
  * ordered workspace).  The tensor cores read the codes decoded to bf16,
- * which is exact for every E4M3 value.  All pointers are device memory
+ * which is exact for every E4M3 value.  Scales must be finite with
+ * |k_scale| * scale < 177 (any usable logit range).  All pointers are device memory
  * owned by the caller; q, k8, v8, out 16-byte aligned.  Returns RA_OK,
  * RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA or RA_ERR_OOM.
  */

@@ -46,8 +46,6 @@
 #include <cstdlib>
 #include <cstring>
 
-#include <cuda_fp8.h>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -69,6 +67,13 @@ constexpr float kSlackSum = 256.f;
 #define RA_EXP2_POLY_MASK 0x00
 #endif
 constexpr int kExp2PolyMask = RA_EXP2_POLY_MASK;
+// FP8-KV kernel ring depths at d = 128 (bf16 slots, FP8 slots).
+#ifndef RA_KV8_NSLOT
+#define RA_KV8_NSLOT 4
+#endif
+#ifndef RA_KV8_NSLOT8
+#define RA_KV8_NSLOT8 4
+#endif
 
 // Register split of the two-query-tile kernel (384 threads at 168 registers).
 constexpr int kLaunchRegs = 168;
@@ -293,15 +298,21 @@ __device__ __forceinline__ void warp_arrive_after_tc(uint32_t bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
-// Four E4M3 codes (bytes of w, lowest address first) to two bf16x2 words.
-// Every E4M3 value, subnormals included, is exact in f16 and in bf16.
+// Four E4M3 codes (bytes of w, lowest address first) to two bf16x2 words
+// holding each code's value times 2^-120 (kFp8Bias), with integer byte moves
+// only.  An E4M3 code s.eeee.mmm placed in a bf16 word as s.0000eeee.mmm0000
+// reads as 2^(e-127) (1 + m/8) = 2^-120 * 2^(e-7) (1 + m/8) for e >= 1, and
+// as the subnormal 2^-126 * m/8 = 2^-120 * 2^-6 * m/8 for e = 0: exact for
+// every finite code.  The 2^120 goes back in through the scales.
+constexpr float kFp8Bias = 1.329227995784916e36f;  // 2^120
 __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  const float2 f01 = __half22float2(__half2(h01));
-  const float2 f23 = __half22float2(__half2(h23));
-  lo = pack_bf16x2(f01.x, f01.y);
-  hi = pack_bf16x2(f23.x, f23.y);
+  const uint32_t em = w & 0x7F7F7F7Fu;  // exponent and mantissa of each code
+  const uint32_t sg = w & 0x80808080u;  // sign of each code
+  // Codes 0, 1 -> bf16 halves of lo; codes 2, 3 -> halves of hi.  Exponent
+  // and mantissa land in the low byte of each half and move up 4 bits; the
+  // sign byte lands in the high byte (bit 7 -> bit 15).
+  lo = __byte_perm(em, 0, 0x4140) * 16u + __byte_perm(sg, 0, 0x1404);
+  hi = __byte_perm(em, 0, 0x4342) * 16u + __byte_perm(sg, 0, 0x3424);
 }
 
 // Decode one FP8 tile (128 keys x D codes, row-major, as the TMA copy left it)
@@ -310,26 +321,29 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint3
 // row r stored at chunk j ^ (r mod 8).  Thread ct of the converter warpgroup
 // takes every 128th 16-code chunk; a warp reads 512 contiguous bytes.
 template <int D>
-__device__ __forceinline__ void convert_fp8_tile(const uint8_t* src, uint32_t dst, int ct) {
+__device__ __forceinline__ void convert_fp8_tile(const uint8_t* src, uint8_t* dst, int ct) {
   constexpr int kChunksPerRow = D / 16;
+  constexpr int kPerThread = kTileN * kChunksPerRow / 128;
+  // All of this thread's loads first, so their latencies overlap.
+  uint4 w[kPerThread];
 #pragma unroll
-  for (int i = 0; i < kTileN * kChunksPerRow / 128; ++i) {
+  for (int i = 0; i < kPerThread; ++i) {
+    const int c = ct + 128 * i;
+    w[i] = *reinterpret_cast<const uint4*>(src + (c / kChunksPerRow) * D + (c % kChunksPerRow) * 16);
+  }
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
     const int c = ct + 128 * i;
     const int r = c / kChunksPerRow, cc = c % kChunksPerRow;
-    const uint4 w = *reinterpret_cast<const uint4*>(src + r * D + cc * 16);
-    uint32_t o[8];
-    e4m3x4_to_bf16x4(w.x, o[0], o[1]);
-    e4m3x4_to_bf16x4(w.y, o[2], o[3]);
-    e4m3x4_to_bf16x4(w.z, o[4], o[5]);
-    e4m3x4_to_bf16x4(w.w, o[6], o[7]);
+    uint4 o0, o1;
+    e4m3x4_to_bf16x4(w[i].x, o0.x, o0.y);
+    e4m3x4_to_bf16x4(w[i].y, o0.z, o0.w);
+    e4m3x4_to_bf16x4(w[i].z, o1.x, o1.y);
+    e4m3x4_to_bf16x4(w[i].w, o1.z, o1.w);
     const int j0 = (cc % 4) * 2;  // 16 codes = 32 bytes of bf16: chunks j0, j0 + 1
-    const uint32_t row = dst + (cc / 4) * (kTileN * 128) + r * 128;
-    const uint32_t a0 = row + ((uint32_t)(j0 ^ (r & 7)) << 4);
-    const uint32_t a1 = row + ((uint32_t)((j0 + 1) ^ (r & 7)) << 4);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a0), "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
-                 : "memory");
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
-                 : "memory");
+    uint8_t* row = dst + (cc / 4) * (kTileN * 128) + r * 128;
+    *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) << 4)) = o0;
+    *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) << 4)) = o1;
   }
 }
 
@@ -638,7 +652,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
           const uint32_t slot8 = f % NSLOT8, slot = f % NSLOT;
           if (!(ok = mbar_wait(BAR_F8_FULL(slot8), (f / NSLOT8) & 1u, abort_flag))) break;
           if (!(ok = mbar_wait(BAR_KV_EMPTY(slot), ((f / NSLOT) & 1u) ^ 1u, abort_flag))) break;
-          convert_fp8_tile<D>(smem + L::kF8Off + slot8 * L::kF8Bytes, sbase + L::kKVOff + slot * L::kTileBytes, ct);
+          convert_fp8_tile<D>(smem + L::kF8Off + slot8 * L::kF8Bytes, smem + L::kKVOff + slot * L::kTileBytes, ct);
           // The bf16 tile is read by the tensor cores (async proxy).
           fence_proxy_async_smem();
           __syncwarp();
@@ -672,7 +686,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
     // folded into the exponent's FMA; otherwise scores are scaled first.
     // FP8 KV cache: k = code * k_scale folds into the score scale, v = code *
     // v_scale into the final normalisation.
-    const float k_mul = kKV8 ? p.k_scale[b * p.Hkv + hk] : 1.f;
+    // The decoded tiles hold code values times 2^-120: the scores come back
+    // up through the score scale (finite while scale * k_scale < 177), the
+    // output through the epilogue (O * 2^120 first, then v_scale / l).
+    const float k_mul = kKV8 ? p.k_scale[b * p.Hkv + hk] * kFp8Bias : 1.f;
     const float v_mul = kKV8 ? p.v_scale[b * p.Hkv + hk] : 1.f;
     const float scale_l2 = p.scale_log2 * k_mul;
     const bool fold = scale_l2 > 0.f;
@@ -844,6 +861,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
           if (n > 0) {
             tmem_ld32(o_tmem + c * 32, r);
             tc_wait_ld();
+            if constexpr (kKV8) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] *= kFp8Bias;
+            }
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = 0.f;
@@ -1046,8 +1067,8 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
       if (mode == kModeFinal) return launch_cfg<64, 1, 6, kModeFinal, 8>(prm, grid, st);
       return launch_cfg<64, 1, 6, kModeSplit, 8>(prm, grid, st);
     }
-    if (mode == kModeFinal) return launch_cfg<128, 1, 4, kModeFinal, 4>(prm, grid, st);
-    return launch_cfg<128, 1, 4, kModeSplit, 4>(prm, grid, st);
+    if (mode == kModeFinal) return launch_cfg<128, 1, RA_KV8_NSLOT, kModeFinal, RA_KV8_NSLOT8>(prm, grid, st);
+    return launch_cfg<128, 1, RA_KV8_NSLOT, kModeSplit, RA_KV8_NSLOT8>(prm, grid, st);
   }
   if (a.d == 64) {
     if (two) { RA_LAUNCH(64, 2, 8) } else { RA_LAUNCH(64, 1, 8) }

@@ -83,6 +83,10 @@ CONFIGS = {
     "5d8f8": Workload("cache_idx_decode_fp8kv_Nq8_Nkv262144", B=4, Hq=32, Hkv=8, N_q=8, N_kv=262144, d=128,
                       dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5500,
                       kv_dtype="fp8"),
+    # Quarter-length FP8 cache (0.54 GB of codes) for profiler captures.
+    "5d1f8s": Workload("cache_idx_decode_fp8kv_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
+                       dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5600,
+                       kv_dtype="fp8"),
     "5d1s": Workload("cache_idx_decode_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
                      dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5300),
 }
