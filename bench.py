@@ -85,6 +85,8 @@ def flops_of(w: workloads.Workload) -> float:
 
     Causal prefill counts half of the square (2*B*Hq*N^2*d); an incremental
     query block counts its exact visible pairs."""
+    if w.window >= 0:
+        return 4.0 * w.d * w.B * w.Hq * window_anchor_pairs(w.N_q, w.window, w.anchor_period)
     if w.cache_idx < 0:
         pairs = w.N_q * w.N_kv * (0.5 if w.causal else 1.0)
     elif w.causal:
@@ -92,6 +94,20 @@ def flops_of(w: workloads.Workload) -> float:
     else:
         pairs = float(w.N_q * w.N_kv)
     return 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def window_anchor_pairs(n: int, window: int, period: int) -> float:
+    """Visible (query, key) pairs of the window-and-anchor mask: each row's
+    window [max(0, i - W), i], plus its anchors a, a - 1 (a > 0) and a + A
+    (a < n - A) where they fall outside that window."""
+    i = np.arange(n, dtype=np.int64)
+    lo = np.maximum(0, i - window)
+    a = i - i % period
+    count = (i - lo + 1).astype(np.float64)
+    count += (a < lo)
+    count += (a > 0) & (a - 1 < lo)
+    count += a < n - period
+    return float(count.sum())
 
 
 def hbm_bytes_of(w: workloads.Workload) -> float:
@@ -198,6 +214,10 @@ def run_ours(args, w, rank, world, device):
     if fp8:
         def fn(q_, k_, v_, **kw):
             return R.ring_attn_fwd_fp8kv(q_, k_, v_, k_sc, v_sc, **kw)
+    elif w.window >= 0:
+        def fn(q_, k_, v_, *, causal, P, chunk, cache_idx, scale, out, lse, stream):
+            return R.ring_attn_fwd_window_anchor(q_, k_, v_, window=w.window, anchor_period=w.anchor_period, P=P,
+                                                 chunk=chunk, scale=scale, out=out, lse=lse, stream=stream)
     else:
         fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
 
@@ -351,9 +371,17 @@ def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
         qs = q[:, r0:r0 + nr, h:h + 1].double().numpy()
         base = (0 if w.cache_idx < 0 else w.cache_idx) + r0
         t0 = time.perf_counter()
-        oracle.attention_ref(qs, kf[hk][0], kf[hk][1], causal=w.causal, scale=w.scale, cache_idx=base)
+        if w.window >= 0:
+            oracle.attention_window_anchor_ref(q[:, :, h:h + 1].double().numpy(), kf[hk][0], kf[hk][1],
+                                               window=w.window, anchor_period=w.anchor_period, scale=w.scale,
+                                               rows=np.arange(r0, r0 + nr))
+        else:
+            oracle.attention_ref(qs, kf[hk][0], kf[hk][1], causal=w.causal, scale=w.scale, cache_idx=base)
         elapsed += time.perf_counter() - t0
-        vis = [(base + i + 1) if w.causal else w.N_kv for i in range(nr)]
+        if w.window >= 0:
+            vis = [min(r0 + i, w.window) + 1 + 2 for i in range(nr)]
+        else:
+            vis = [(base + i + 1) if w.causal else w.N_kv for i in range(nr)]
         flops += 4.0 * w.d * w.B * sum(min(x, w.N_kv) for x in vis)
         rows_done += nr
         if time.perf_counter() - t_start > 4 * budget_s:
@@ -425,7 +453,10 @@ def main():
     # forward's size instead of two); the dQ kernel's recomputation of S and
     # dP is not counted.
     flops = flops_of(w) * (2.5 if bwd else 1.0)
-    config = {"workload": w.name, "kv_cache": "fp8 e4m3 + per-head scales" if w.kv_dtype == "fp8" else w.dtype,
+    config = {"workload": w.name,
+              "mask": (f"window {w.window} + anchors every {w.anchor_period}" if w.window >= 0 else
+                       "causal" if w.causal else "none"),
+              "kv_cache": "fp8 e4m3 + per-head scales" if w.kv_dtype == "fp8" else w.dtype,
               "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
               "causal": w.causal, "P": w.P, "chunk": w.chunk, "cache_idx": w.cache_idx, "k_scale": w.k_scale,
               "global_batch": w.B * world, "l2": "inputs larger than the 126 MB L2, no flush"

@@ -190,6 +190,23 @@ int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const flo
                         int64_t cache_idx, float scale, void* stream);
 
 /*
+ * ring_attn_fwd_window_anchor -- ring_attn_fwd (bf16, square prefill,
+ * N_q == N_kv == N) under the sparse mask of "Ring Attention: the secret of
+ * million-token context" §4.3 instead of the causal one: query i attends to
+ * its local window, keys max(0, i - window) .. i, and to the anchors of its
+ * period A = anchor_period: with a = floor(i / A) * A, the keys a, a - 1
+ * (a > 0) and a + A (when a < N - A; that key lies after i).  Tiles that
+ * hold none of a row block's keys are skipped.  The result is exact
+ * attention under that mask (approximate attention with respect to the
+ * full causal one).  window in [0, N]; anchor_period > 0 and a multiple of
+ * 256.  Layouts, chunk / P, scale, ownership and status codes as
+ * ring_attn_fwd.
+ */
+int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, void* out, float* lse,
+                                int B, int Hq, int Hkv, int64_t N, int d, int64_t chunk, int P,
+                                int64_t window, int64_t anchor_period, float scale, void* stream);
+
+/*
  * ring_attn_bwd_block_step -- the backward of one ring visit: adds, in
  * place, the share of dq, dk, dv that comes from the pairs of query chunk
  * q_chunk [B, Lq, Hq, d] (global positions q_off + t) and KV chunk

@@ -118,26 +118,57 @@ struct Sm100Params {
   int tpt;     // tokens per tile: 128 / gpack
   const float* k_scale;  // FP8 KV cache: [B, Hkv] dequantisation scales
   const float* v_scale;
+  int wa_window;  // window-and-anchor mask: window W (keys i - W .. i) ...
+  int wa_period;  // ... and anchor period A; 0: no such mask
 };
+
+// The window-and-anchor sparse mask as seen by one CTA: keys [lo, hi] hold
+// the local windows of its query rows, and a0, am1, ap its anchor keys
+// (a, a - 1, a + A; -1 when absent).  All of a CTA's rows share one anchor
+// period (A is a multiple of its row span).
+// It lives in shared memory (written once per CTA), so the roles' cursors
+// carry no registers for it; kernels without the mask never touch it.
+struct WinAnchor {
+  int W, lo, hi, a0, am1, ap;
+};
+__shared__ WinAnchor s_wa;
+
+__device__ __forceinline__ bool wa_has_anchor(int k0, int kend) {
+  return (s_wa.a0 >= k0 && s_wa.a0 < kend) || (s_wa.am1 >= k0 && s_wa.am1 < kend) ||
+         (s_wa.ap >= k0 && s_wa.ap < kend);
+}
+// Does any row of the CTA see a key in [k0, kend)?
+template <bool WA>
+__device__ __forceinline__ bool wa_live(int k0, int kend) {
+  if constexpr (!WA) return true;
+  return (kend - 1 >= s_wa.lo && k0 <= s_wa.hi) || wa_has_anchor(k0, kend);
+}
 
 // The sequence of KV tiles one CTA visits: chunks in ring order from `home`,
 // 128-key tiles inside each chunk, keys clipped to [0, lim).  Indices are
 // k-buffer rows; the host caps buffers well below 2^31 rows, so 32 bits hold
 // every sum formed here.
+//
+// Under the window-and-anchor mask the cursor yields only tiles some row of
+// the CTA sees (chunks and tiles outside the windows and anchors are
+// skipped); every role walks the same cursor, so they stay in step.
+template <bool WA>
 struct KvCursor {
   int chunk, lim, P, home, s, s_end;
   int k0, kend, cend;
 
+  // First live tile of chunk step s or a later one.
   __device__ __forceinline__ void load_chunk() {
     while (s < s_end) {
       const int c = (home + s) % P;
       const int cb = c * chunk;
       const int ce = min(cb + chunk, lim);
-      if (cb < ce) {
-        k0 = cb;
+      if (cb < ce && wa_live<WA>(cb, ce)) {
         cend = ce;
-        kend = min(k0 + kTileN, cend);
-        return;
+        for (k0 = cb; k0 < ce; k0 += kTileN) {
+          kend = min(k0 + kTileN, ce);
+          if (wa_live<WA>(k0, kend)) return;
+        }
       }
       ++s;
     }
@@ -153,13 +184,12 @@ struct KvCursor {
   }
   __device__ __forceinline__ bool valid() const { return s < s_end; }
   __device__ __forceinline__ void next() {
-    k0 += kTileN;
-    if (k0 < cend) {
+    for (k0 += kTileN; k0 < cend; k0 += kTileN) {
       kend = min(k0 + kTileN, cend);
-    } else {
-      ++s;
-      load_chunk();
+      if (wa_live<WA>(k0, kend)) return;
     }
+    ++s;
+    load_chunk();
   }
 };
 
@@ -216,11 +246,15 @@ __device__ __forceinline__ QTile make_qtile(int qblk, int t, long long N_q, long
   return q;
 }
 
-__device__ __forceinline__ bool tile_visible(const QTile& q, int k0, int causal) {
+template <bool WA>
+__device__ __forceinline__ bool tile_visible(const QTile& q, int k0, int kend, int causal) {
+  if constexpr (WA) return q.nv > 0 && ((kend - 1 >= q.kmin - s_wa.W && k0 <= q.kmax) || wa_has_anchor(k0, kend));
   return q.nv > 0 && (!causal || k0 <= q.kmax);
 }
 
+template <bool WA>
 __device__ __forceinline__ bool tile_needs_mask(const QTile& q, int k0, int kend, int causal) {
+  if constexpr (WA) return (kend - k0 < kTileN) || k0 < q.kmax - s_wa.W || kend - 1 > q.kmin;
   return (kend - k0 < kTileN) || (causal && kend - 1 > q.kmin);
 }
 
@@ -347,7 +381,7 @@ __device__ __forceinline__ void convert_fp8_tile(const uint8_t* src, uint8_t* ds
   }
 }
 
-template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0>
+template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0, bool WA = false>
 __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
     fwd_sm100_kernel(const __grid_constant__ Sm100Params p) {
   using L = Layout<D, NQT, NSLOT, NSLOT8>;
@@ -411,6 +445,17 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
     if (qt[t].nv > 0) kmax_last = qt[t].kmax;
   int lim = (int)p.N_kv;
   if (p.causal) lim = max(0, min(lim, kmax_last + 1));
+  if (WA && threadIdx.x == 0) {
+    // Square prefill: query t sits at position t, key j at j.  Published by
+    // the set-up barrier below.
+    s_wa.W = p.wa_window;
+    s_wa.lo = max(0, qt[0].kmin - p.wa_window);
+    s_wa.hi = kmax_last;
+    const int a = (qt[0].tok0 / p.wa_period) * p.wa_period;
+    s_wa.a0 = a;
+    s_wa.am1 = a > 0 ? a - 1 : -1;
+    s_wa.ap = (long long)a + p.wa_period < p.N_kv ? a + p.wa_period : -1;
+  }
   const long long first_rel = qk_delta + qt[0].tok0;
   const int home = first_rel > 0 ? (int)min((long long)(p.P - 1), first_rel / p.chunk) : 0;
   const int s_begin = sigma * p.steps_per_split;
@@ -476,7 +521,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
           tma_load_4d(sbase + L::kQOff + t * L::kTileBytes + hf * (kTileM * 128), &p.tm_q, BAR_Q(), hf * 64, h,
                       qt[t].tok0, b);
       }
-      KvCursor cur;
+      KvCursor<WA> cur;
       cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t issued = 0;  // slot fills issued (2 per KV tile)
       bool ok = true;
@@ -541,7 +586,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
         n_seen[t] = 0;
         o_live[t] = (MODE == kModeState);
       }
-      KvCursor cur;
+      KvCursor<WA> cur;
       cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t j = 0;  // KV tile index
       if (ok && cur.valid()) {
@@ -550,7 +595,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
         if (ok) {
 #pragma unroll
           for (int t = 0; t < NQT; ++t)
-            if (tile_visible(qt[t], cur.k0, p.causal)) {
+            if (tile_visible<WA>(qt[t], cur.k0, cur.kend, p.causal)) {
               mma_qk<D, 0, 2>(tmem + 128 * t, qdesc[t], kv_addr(0));
               tc_commit(BAR_S(t));
             }
@@ -567,7 +612,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
       //                        S columns, after PV has read P.
 
       while (ok && cur.valid()) {
-        KvCursor nxt = cur;
+        KvCursor<WA> nxt = cur;
         nxt.next();
         const bool has_next = nxt.valid();
         const uint32_t vfill = 2 * j + 1, kfill = 2 * j + 2;
@@ -585,8 +630,8 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
         };
 #pragma unroll
         for (int t = 0; t < NQT && ok; ++t) {
-          const bool vc = tile_visible(qt[t], cur.k0, p.causal);
-          const bool vn = has_next && tile_visible(qt[t], nxt.k0, p.causal);
+          const bool vc = tile_visible<WA>(qt[t], cur.k0, cur.kend, p.causal);
+          const bool vn = has_next && tile_visible<WA>(qt[t], nxt.k0, nxt.kend, p.causal);
           if (vc) {
             const uint32_t par = n_seen[t] & 1u;
             ++n_seen[t];
@@ -643,7 +688,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
     if constexpr (kKV8) {
       reg_dealloc<kRegsConvert8>();
       const int ct = (int)threadIdx.x - (128 + 128 * NQT);
-      KvCursor cur;
+      KvCursor<WA> cur;
       cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t f = 0;  // fills converted, in the producer's order (K_j, V_j, ...)
       bool ok = true;
@@ -720,12 +765,12 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
     const float m2_in = m2;
     float m_true = m2;  // true running max (kept for the state epilogue)
 
-    KvCursor cur;
+    KvCursor<WA> cur;
     cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
     uint32_t n = 0;
     bool ok = true;
     while (warp_active && cur.valid()) {
-      if (tile_visible(q, cur.k0, p.causal)) {
+      if (tile_visible<WA>(q, cur.k0, cur.kend, p.causal)) {
         if (!mbar_wait(BAR_S(t), n & 1u, abort_flag)) {
           ok = false;
           break;
@@ -745,8 +790,33 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] *= scale_l2;
         }
-        const bool masked = tile_needs_mask(q, cur.k0, cur.kend, p.causal);
-        if (masked) {
+        const bool masked = tile_needs_mask<WA>(q, cur.k0, cur.kend, p.causal);
+        if (WA && masked) {
+          // This row's window [pos - W, pos] and the CTA's anchors, inside
+          // the keys of this tile (tile-relative).
+          const int kvis = cur.kend - cur.k0;
+          const int pos = q.kmin + tl;
+          const int kf = max(0, pos - s_wa.W - cur.k0);
+          const int kl = min(kvis - 1, pos - cur.k0);
+          // 128 visibility bits for this row: the window [kf, kl], then
+          // the anchors that fall inside the tile's keys.
+          uint32_t vm[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = min(max(kf - 32 * w, 0), 32), hi = min(max(kl + 1 - 32 * w, 0), 32);
+            vm[w] = hi > lo ? (uint32_t)((((1ull << hi) - 1ull) >> lo) << lo) : 0u;
+          }
+          const int xs[3] = {s_wa.a0 - cur.k0, s_wa.am1 - cur.k0, s_wa.ap - cur.k0};
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int x = xs[i];
+            const bool in = (i == 0 || (i == 1 ? s_wa.am1 >= 0 : s_wa.ap >= 0)) && x >= 0 && x < kvis;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) vm[w] |= (in && (x >> 5) == w) ? (1u << (x & 31)) : 0u;
+          }
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = ((vm[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+        } else if (masked) {
           const int kvis = cur.kend - cur.k0;  // keys inside the chunk / range
           // Last key (tile-relative) this row sees under causal masking.
           const long long kc = p.causal ? (long long)q.kmin + tl - cur.k0 : (long long)kTileN;
@@ -924,10 +994,10 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
   if (warp == 2) tmem_dealloc(tmem, L::kTmemCols);
 }
 
-template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0>
+template <int D, int NQT, int NSLOT, int MODE, int NSLOT8 = 0, bool WA = false>
 cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) {
   using L = Layout<D, NQT, NSLOT, NSLOT8>;
-  auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE, NSLOT8>;
+  auto kern = fwd_sm100_kernel<D, NQT, NSLOT, MODE, NSLOT8, WA>;
   static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
   constexpr int kThreads = 128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0);
   if constexpr (NQT == 2 || NSLOT8 > 0) {
@@ -1051,6 +1121,8 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   }
   prm.tpt = geo.tpt;
   prm.n_qblk = geo.n_qblk;
+  prm.wa_window = a.wa_window;
+  prm.wa_period = a.wa_period;
   const bool two = geo.two;
   const long long grid = geo.ctas_per_split * prm.S;
   // K/V ring depth: as many 128-key slots as shared memory allows
@@ -1060,6 +1132,16 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
     case kModeFinal: return launch_cfg<D_, NQT_, NS_, kModeFinal>(prm, grid, st); \
     case kModeSplit: return launch_cfg<D_, NQT_, NS_, kModeSplit>(prm, grid, st); \
     default: return launch_cfg<D_, NQT_, NS_, kModeState>(prm, grid, st);        \
+  }
+  if (a.wa_period > 0) {
+    // Window-and-anchor mask: square prefill, one launch.
+    if (mode != kModeFinal) return cudaErrorInvalidValue;
+    if (a.d == 64) {
+      if (two) return launch_cfg<64, 2, 8, kModeFinal, 0, true>(prm, grid, st);
+      return launch_cfg<64, 1, 8, kModeFinal, 0, true>(prm, grid, st);
+    }
+    if (two) return launch_cfg<128, 2, 5, kModeFinal, 0, true>(prm, grid, st);
+    return launch_cfg<128, 1, 6, kModeFinal, 0, true>(prm, grid, st);
   }
   if (a.kv8) {
     // One query tile, bf16 ring, FP8 ring (d=128: 32 + 4 x 32 + 4 x 16 = 224 KB).

@@ -53,6 +53,8 @@ struct ProblemArgs {
   int kv8;          // 1: k and v are FP8 E4M3 codes, dequantised by k_scale / v_scale [B, Hkv]
   const float* k_scale;
   const float* v_scale;
+  int wa_window;    // window-and-anchor mask (square prefill, causal = 0): window W and
+  int wa_period;    // anchor period A (a multiple of 256); wa_period = 0: no such mask
 };
 
 // Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.

@@ -244,6 +244,29 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
   return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd");
 }
 
+int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                                int Hkv, int64_t N, int d, int64_t chunk, int P, int64_t window,
+                                int64_t anchor_period, float scale, void* stream) {
+  if (window < 0 || window > kMaxTokens || anchor_period <= 0 || anchor_period % 256 != 0 ||
+      anchor_period > kMaxTokens)
+    return RA_ERR_INVALID_ARG;
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N, N, d, 0, chunk, P, -1, scale, true);
+  if (r != RA_OK) return r;
+  if (B == 0 || N == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  ProblemArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.N_q = N; a.N_kv = N;
+  a.q_pos0 = 0; a.k_pos0 = 0;
+  a.causal = 0; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0; a.S = 1;
+  a.wa_window = (int)window;
+  a.wa_period = (int)anchor_period;
+  return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd_window_anchor");
+}
+
 int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const float* k_scale, const float* v_scale,
                         void* out, float* lse, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
                         int64_t chunk, int P, int64_t cache_idx, float scale, void* stream) {

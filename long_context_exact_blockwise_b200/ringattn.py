@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
-    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_fwd_fp8kv", "ring_attn_bwd", "ring_attn_bwd_block_step", "ring_attn_block_step", "ring_attn_finalize",
+    "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_fwd_fp8kv", "ring_attn_fwd_window_anchor", "ring_attn_bwd", "ring_attn_bwd_block_step", "ring_attn_block_step", "ring_attn_finalize",
     "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
@@ -54,6 +54,7 @@ _SIGS = {
     "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_fwd_window_anchor": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _i, _l, _i, _l, _l, _f, _p],
     "ring_attn_fwd_fp8kv": [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
     "ring_attn_bwd_block_step": [_p, _p, _p, _p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _p],
@@ -207,6 +208,29 @@ def ring_attn_fwd_fp8kv(q, k8, v8, k_scale, v_scale, *, causal: bool, P: int, ch
                                  B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)), int(chunk), int(P), ci, sc,
                                  _stream(stream, q.device))
     _check(st, "ring_attn_fwd_fp8kv")
+    return out, lse
+
+
+def ring_attn_fwd_window_anchor(q, k, v, *, window: int, anchor_period: int, P: int = 1,
+                                chunk: Optional[int] = None, scale: Optional[float] = None, out=None, lse=None,
+                                stream=None):
+    """bf16 square prefill under the window-and-anchor sparse mask -> (out, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16)
+    B, N, Hq, d = q.shape
+    _, N_kv, Hkv, _ = k.shape
+    if N_kv != N or v.shape != k.shape:
+        raise ValueError("the window-and-anchor mask needs N_q == N_kv")
+    chunk = N // P if chunk is None else chunk
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _need(out, "out", torch.bfloat16)
+    _need(lse, "lse", torch.float32)
+    st = lib.ring_attn_fwd_window_anchor(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                                         int(chunk), int(P), int(window), int(anchor_period), sc,
+                                         _stream(stream, q.device))
+    _check(st, "ring_attn_fwd_window_anchor")
     return out, lse
 
 

@@ -149,3 +149,14 @@ def test_fp8kv_validation():
     assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG
     bad = list(ok_args); bad[14] = 100  # N_kv != P * chunk
     assert L.ring_attn_fwd_fp8kv(*bad) == ra.RA_ERR_INVALID_ARG
+
+
+def test_window_anchor_validation():
+    ra = _lib()
+    L = ra.lib
+    # q, k, v, out, lse, B, Hq, Hkv, N, d, chunk, P, window, anchor_period, scale, stream
+    ok_args = [FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 256, 4, 64, 256, 0.1, None]
+    assert L.ring_attn_fwd_window_anchor(*ok_args) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
+    for i, val in ((12, -1), (13, 0), (13, 100), (13, 384), (9, 96), (10, 100)):
+        bad = list(ok_args); bad[i] = val
+        assert L.ring_attn_fwd_window_anchor(*bad) == ra.RA_ERR_INVALID_ARG, (i, val)

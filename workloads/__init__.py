@@ -44,6 +44,8 @@ class Workload:
     k_scale: float = 1.0  # exact power-of-two multiplier applied to K before the cast
     seed: int = 0         # q uses seed, k seed+1, v seed+2
     kv_dtype: str = "bf16"  # "fp8": the KV cache is stored as FP8 E4M3 codes with scales (make_fp8_kv)
+    window: int = -1        # >= 0: window-and-anchor sparse mask (square prefill) with this window ...
+    anchor_period: int = 0  # ... and this anchor period
 
     @property
     def scale(self) -> float:
@@ -83,6 +85,11 @@ CONFIGS = {
     "5d8f8": Workload("cache_idx_decode_fp8kv_Nq8_Nkv262144", B=4, Hq=32, Hkv=8, N_q=8, N_kv=262144, d=128,
                       dtype="bf16", causal=True, P=64, chunk=4096, cache_idx=262144 - 8, seed=5500,
                       kv_dtype="fp8"),
+    # The GQA prefill under the window-and-anchor sparse mask (16K-token window,
+    # an anchor every 4096 tokens).
+    "wa3": Workload("window_anchor_prefill_N131072_W16384_A4096", B=1, Hq=32, Hkv=8, N_q=131072, N_kv=131072,
+                    d=128, dtype="bf16", causal=False, P=16, chunk=8192, seed=3100, window=16384,
+                    anchor_period=4096),
     # Quarter-length FP8 cache (0.54 GB of codes) for profiler captures.
     "5d1f8s": Workload("cache_idx_decode_fp8kv_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
                        dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5600,
@@ -97,7 +104,8 @@ def workload(key) -> Workload:
 
 
 def small(B=1, Hq=2, Hkv=1, N_q=200, N_kv=None, d=64, dtype="bf16", causal=True, P=2,
-          chunk=None, cache_idx=-1, k_scale=1.0, seed=7, name="small", kv_dtype="bf16") -> Workload:
+          chunk=None, cache_idx=-1, k_scale=1.0, seed=7, name="small", kv_dtype="bf16", window=-1,
+          anchor_period=0) -> Workload:
     """A small problem for parity tests (sizes the CPU oracle finishes quickly)."""
     if N_kv is None:
         N_kv = N_q if cache_idx < 0 else cache_idx + N_q
@@ -105,7 +113,7 @@ def small(B=1, Hq=2, Hkv=1, N_q=200, N_kv=None, d=64, dtype="bf16", causal=True,
         chunk = N_kv // P
     return Workload(name, B=B, Hq=Hq, Hkv=Hkv, N_q=N_q, N_kv=N_kv, d=d, dtype=dtype,
                     causal=causal, P=P, chunk=chunk, cache_idx=cache_idx, k_scale=k_scale,
-                    seed=seed, kv_dtype=kv_dtype)
+                    seed=seed, kv_dtype=kv_dtype, window=window, anchor_period=anchor_period)
 
 
 def _randn(shape, seed: int, device, mult: float, dtype: torch.dtype) -> torch.Tensor:
