@@ -1075,6 +1075,7 @@ Sm100Geometry sm100_geometry(const ProblemArgs& a, int mode) {
 
 cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   if (a.B <= 0 || a.N_q <= 0) return cudaSuccess;
+  if (decode_rows(a, mode) > 0) return launch_decode_sm100(a, mode, st);
   const Sm100Geometry geo = sm100_geometry(a, mode);
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));

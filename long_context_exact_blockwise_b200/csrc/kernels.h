@@ -60,6 +60,12 @@ struct ProblemArgs {
 // Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.
 cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
 
+// Keys-on-M decode kernel (d = 128, incremental queries with G * N_q <= 32
+// rows per KV head): rows per block it would use (16 or 32; 0 = not
+// applicable), and its launcher.  launch_fwd_sm100 routes such problems to it.
+int decode_rows(const ProblemArgs& a, int mode);
+cudaError_t launch_decode_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
+
 // CTA geometry the tensor-core path uses for a problem: query heads packed
 // per tile (gpack), tokens per tile, one or two query tiles per CTA, and the
 // number of CTAs per KV split.

@@ -14,6 +14,7 @@
 // The kernels and their launchers (one translation unit: the status word is
 // shared without relocatable device code).
 #include "fwd_sm100.cuh"
+#include "decode_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "fwd_simt.cuh"
 #include "merge.cuh"

@@ -90,6 +90,9 @@ CONFIGS = {
     "wa3": Workload("window_anchor_prefill_N131072_W16384_A4096", B=1, Hq=32, Hkv=8, N_q=131072, N_kv=131072,
                     d=128, dtype="bf16", causal=False, P=16, chunk=8192, seed=3100, window=16384,
                     anchor_period=4096),
+    # Quarter-length 8-token decode (1.07 GB of K/V) for profiler captures.
+    "5d8s": Workload("cache_idx_decode_Nq8_Nkv65536", B=4, Hq=32, Hkv=8, N_q=8, N_kv=65536, d=128,
+                     dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 8, seed=5700),
     # Quarter-length FP8 cache (0.54 GB of codes) for profiler captures.
     "5d1f8s": Workload("cache_idx_decode_fp8kv_Nq1_Nkv65536", B=4, Hq=32, Hkv=8, N_q=1, N_kv=65536, d=128,
                        dtype="bf16", causal=True, P=16, chunk=4096, cache_idx=65536 - 1, seed=5600,
