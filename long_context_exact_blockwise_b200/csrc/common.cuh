@@ -71,6 +71,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete may
+// stay suspended up to hint_ns (it resumes when the phase completes), so a
+// long wait costs few issue slots.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for waits off the latency-critical path: suspended rather than
+// polling, with the same wall-clock bound and abort handling.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  constexpr uint32_t kHintNs = 20000;
+  if (mbar_try_wait_hint(bar, parity, kHintNs)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, kHintNs)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(&g_status, (int)RA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Wait for the phase with the given parity to complete, with a wall-clock
 // bound.  Returns false (after flagging the CTA and the device status word)
 // if the bound expires, or if another thread of the CTA already aborted.

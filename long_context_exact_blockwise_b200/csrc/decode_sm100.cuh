@@ -19,13 +19,15 @@
 //   warp 1       MMA issuer: S^T_j into one of two TMEM buffers (two tiles
 //                ahead), O^T += V^T_j P^T_j once P^T_j is in shared memory.
 //   warp 2       TMEM allocator.
-//   warps 4-7    softmax: thread = key of the tile (TMEM lane).  Per tile:
-//                the column maxima over the 128 keys (warp reductions, then
-//                the four warps through shared memory), the running base
-//                per row (rescaling O^T in TMEM when it moves past a slack),
-//                P^T as bf16 into shared memory, per-thread partial row sums.
-//                Epilogue: thread = channel d of O^T.
-//   warps 8-11   (FP8 cache) converters, as in fwd_sm100.cuh.
+//   warps 4-11   softmax: thread = key of the tile (TMEM lane); warp w takes
+//                lane quarter w mod 4 and half of the NR row columns, so two
+//                warps per SM sub-partition hide each other's latency.  Per
+//                tile: the column maxima over the 128 keys (warp reductions,
+//                then the four lane quarters through shared memory), the
+//                running base per row (rescaling O^T in TMEM when it moves
+//                past a slack), P^T as bf16 into shared memory, per-thread
+//                partial row sums.  Epilogue: thread = channel d of O^T.
+//   warps 12-15  (FP8 cache) converters, as in fwd_sm100.cuh.
 // Every mbarrier wait is bounded; the warpgroup's exchange of column maxima
 // also goes through an mbarrier, so an expired wait anywhere unwinds the CTA.
 #pragma once
@@ -51,21 +53,35 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
       : "r"(taddr));
 }
 
-template <int NR>
-__device__ __forceinline__ void tmem_ld_nr(uint32_t taddr, float (&r)[NR]) {
-  static_assert(NR == 16 || NR == 32, "row block of 16 or 32");
-  if constexpr (NR == 16)
-    tmem_ld16(taddr, r);
-  else
-    tmem_ld32(taddr, r);
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&r)[8]) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(u[0]),
+               "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+               : "memory");
 }
 
-template <int NR>
-__device__ __forceinline__ void tmem_st_nr(uint32_t taddr, const float (&r)[NR]) {
-  if constexpr (NR == 16)
-    tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(r));
+// CH = 8 or 16 columns of this thread's lane.
+template <int CH>
+__device__ __forceinline__ void tmem_ld_ch(uint32_t taddr, float (&r)[CH]) {
+  static_assert(CH == 8 || CH == 16, "8 or 16 columns per warp");
+  if constexpr (CH == 8)
+    tmem_ld8(taddr, r);
   else
-    tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(r));
+    tmem_ld16(taddr, r);
+}
+template <int CH>
+__device__ __forceinline__ void tmem_st_ch(uint32_t taddr, const float (&r)[CH]) {
+  if constexpr (CH == 8)
+    tmem_st8(taddr, r);
+  else
+    tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(r));
 }
 
 // Floats as signed integers with the same order (non-NaN), for the warp's
@@ -82,6 +98,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
 }
 
 constexpr int kDecD = 128;  // channels (the decode kernel serves d = 128)
+// Work order: KV heads innermost (1, measured faster on the bf16 cache) or
+// splits innermost (0).
+#ifndef RA_DEC_HEADS_INNER
+#define RA_DEC_HEADS_INNER 1
+#endif
+// CTAs per SM the decode kernel is compiled for.
+#ifndef RA_DEC_MINB
+#define RA_DEC_MINB 1
+#endif
+// Ring depth of the 16-row bf16 configuration.
+#ifndef RA_DEC_NSLOT
+#define RA_DEC_NSLOT 6
+#endif
+// Ring depths of the 16-row FP8 configuration (bf16 slots, FP8 slots).
+#ifndef RA_DEC8_NSLOT
+#define RA_DEC8_NSLOT 5
+#endif
+#ifndef RA_DEC8_NSLOT8
+#define RA_DEC8_NSLOT8 3
+#endif
 
 template <int NR, int NSLOT, int NSLOT8>
 struct DecLayout {
@@ -93,8 +129,8 @@ struct DecLayout {
   static constexpr int kKVOff = 1024 * ((kQBytes + 1023) / 1024);
   static constexpr int kPOff = kKVOff + NSLOT * kTileBytes;
   static constexpr int kF8Off = kPOff + 2 * kPBytes;
-  // [3][4 warps][NR] floats: column maxima (two tile-parity buffers), then
-  // the row sums of the epilogue.
+  // [3][NR][4 lane quarters] floats: column maxima (two tile-parity
+  // buffers), then the row sums of the epilogue.
   static constexpr int kRedOff = kF8Off + NSLOT8 * kF8Bytes;
   static constexpr int kBarOff = kRedOff + 3 * 4 * NR * 4;
   // q, kv_full[NSLOT], kv_empty[NSLOT], s[2], p[2], pv[2], red[2], done, sum,
@@ -129,7 +165,7 @@ struct DecParams {
 };
 
 template <int NR, int NSLOT, int MODE, int NSLOT8>
-__global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel(const __grid_constant__ DecParams p) {
+__global__ void __launch_bounds__(NSLOT8 > 0 ? 512 : 384, RA_DEC_MINB) decode_sm100_kernel(const __grid_constant__ DecParams p) {
   using L = DecLayout<NR, NSLOT, NSLOT8>;
   constexpr bool kKV8 = NSLOT8 > 0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -154,7 +190,19 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: splits innermost, then row blocks, KV heads, batch.
+  // ---- work item.
+#if RA_DEC_HEADS_INNER
+  // KV heads innermost: the CTAs of one (batch, split, row block) run side by
+  // side and read neighbouring slices of the same token rows.
+  long long x = blockIdx.x;
+  const int hk = (int)(x % p.Hkv);
+  x /= p.Hkv;
+  const int sigma = (int)(x % p.S);
+  x /= p.S;
+  const int qblk = (int)(x % p.n_qblk);
+  const int b = (int)(x / p.n_qblk);
+#else
+  // Splits innermost, then row blocks, KV heads, batch.
   long long x = blockIdx.x;
   const int sigma = (int)(x % p.S);
   x /= p.S;
@@ -162,6 +210,7 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
   x /= p.n_qblk;
   const int hk = (int)(x % p.Hkv);
   const int b = (int)(x / p.Hkv);
+#endif
   const int tok0 = qblk * p.tpb;
   const int ntok = (int)min((long long)p.tpb, p.N_q - tok0);
   const int nrows = ntok * p.G;
@@ -182,12 +231,12 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR_S(i), 1);
-      mbar_init(BAR_P(i), 4);
+      mbar_init(BAR_P(i), 8);    // one arrival per softmax warp
       mbar_init(BAR_PV(i), 1);
-      mbar_init(BAR_RED(i), 4);
+      mbar_init(BAR_RED(i), 8);
     }
     mbar_init(BAR_DONE, 1);
-    mbar_init(BAR_SUM, 4);
+    mbar_init(BAR_SUM, 8);
     for (int i = 0; i < NSLOT8; ++i) {
       mbar_init(BAR_F8_FULL(i), 1);
       mbar_init(BAR_F8_EMPTY(i), 4);
@@ -203,10 +252,6 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // With a converter warpgroup (384 threads at 168 registers) registers move
-  // to the softmax warpgroup: 128 * (64 + 232 + 96) <= 384 * 168.
-  static_assert(128 * (64 + 232 + 96) <= 384 * 168, "register split exceeds the launch");
-  if (kKV8 && warp < 4) reg_dealloc<64>();
   // TMEM columns: S^T buffers [0, NR) and [NR, 2 NR), O^T [2 NR, 3 NR).
   auto T_S = [&](int i) { return tmem + (uint32_t)(NR * i); };
   const uint32_t T_O = tmem + 2 * NR;
@@ -229,12 +274,12 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
           const CUtensorMap* map = kv == 0 ? &p.tm_k : &p.tm_v;
           if constexpr (kKV8) {
             const uint32_t slot8 = issued % NSLOT8;
-            if (!(ok = mbar_wait(BAR_F8_EMPTY(slot8), ((issued / NSLOT8) & 1u) ^ 1u, abort_flag))) break;
+            if (!(ok = mbar_wait_idle(BAR_F8_EMPTY(slot8), ((issued / NSLOT8) & 1u) ^ 1u, abort_flag))) break;
             mbar_arrive_expect_tx(BAR_F8_FULL(slot8), L::kF8Bytes);
             tma_load_4d(sbase + L::kF8Off + slot8 * L::kF8Bytes, map, BAR_F8_FULL(slot8), 0, hk, cur.k0, b);
           } else {
             const uint32_t slot = issued % NSLOT;
-            if (!(ok = mbar_wait(BAR_KV_EMPTY(slot), ((issued / NSLOT) & 1u) ^ 1u, abort_flag))) break;
+            if (!(ok = mbar_wait_idle(BAR_KV_EMPTY(slot), ((issued / NSLOT) & 1u) ^ 1u, abort_flag))) break;
             mbar_arrive_expect_tx(BAR_KV_FULL(slot), L::kTileBytes);
             for (int hf = 0; hf < 2; ++hf)
               tma_load_4d(sbase + L::kKVOff + slot * L::kTileBytes + hf * (kTileN * 128), map, BAR_KV_FULL(slot),
@@ -249,21 +294,21 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
       for (uint32_t f = issued > kRing ? issued - kRing : 0; f < issued; ++f) {
         volatile int no_abort = 0;
         if constexpr (kKV8)
-          mbar_wait(BAR_F8_FULL(f % NSLOT8), (f / NSLOT8) & 1u, &no_abort);
+          mbar_wait_idle(BAR_F8_FULL(f % NSLOT8), (f / NSLOT8) & 1u, &no_abort);
         else
-          mbar_wait(BAR_KV_FULL(f % NSLOT), (f / NSLOT) & 1u, &no_abort);
+          mbar_wait_idle(BAR_KV_FULL(f % NSLOT), (f / NSLOT) & 1u, &no_abort);
       }
       volatile int no_abort = 0;
-      mbar_wait(BAR_Q, 0, &no_abort);
+      mbar_wait_idle(BAR_Q, 0, &no_abort);
     }
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
-      bool ok = mbar_wait(BAR_Q, 0, abort_flag);
+      bool ok = mbar_wait_idle(BAR_Q, 0, abort_flag);
       tc_fence_after();
       const uint64_t qdesc = smem_desc_sw128(sbase + L::kQOff, 16, 1024);
       auto kv_addr = [&](uint32_t f) { return sbase + L::kKVOff + (f % NSLOT) * L::kTileBytes; };
-      auto full = [&](uint32_t f) { return mbar_wait(BAR_KV_FULL(f % NSLOT), (f / NSLOT) & 1u, abort_flag); };
+      auto full = [&](uint32_t f) { return mbar_wait_idle(BAR_KV_FULL(f % NSLOT), (f / NSLOT) & 1u, abort_flag); };
       // S^T_j = K_j Q^T into buffer j & 1 (K-major A = K tile, K-major B = Q block).
       auto issue_s = [&](uint32_t j) {
         constexpr uint32_t idesc = idesc_bf16_f32(kTileN, NR, 0);
@@ -288,7 +333,7 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
         issue_s(j);
       }
       for (uint32_t j = 0; j < n_tiles && ok; ++j) {
-        if (!(ok = mbar_wait(BAR_P(j & 1), (j >> 1) & 1u, abort_flag))) break;
+        if (!(ok = mbar_wait_idle(BAR_P(j & 1), (j >> 1) & 1u, abort_flag))) break;
         if (!(ok = full(2 * j + 1))) break;
         tc_fence_after();
         // O^T += V^T_j P^T_j: A = V tile as MN-major (d contiguous), B = P^T (K-major).
@@ -312,26 +357,28 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
       }
       tc_commit(BAR_DONE);
       volatile int no_abort = 0;
-      mbar_wait(BAR_DONE, 0, &no_abort);
+      mbar_wait_idle(BAR_DONE, 0, &no_abort);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     // ============================ softmax ============================
-    if constexpr (kKV8) reg_alloc<232>();
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;  // key of the tile; channel d in the epilogue
+    constexpr int CH = NR / 2;                // row columns of this warp
+    const int quad = warp & 3;                // TMEM lane quarter
+    const int c0 = ((warp - 4) >> 2) * CH;    // first row column of this warp
+    const int row = quad * 32 + lane;         // key of the tile; channel d in the epilogue
     const uint32_t lb = (uint32_t)(quad * 32) << 16;
     const float k_mul = kKV8 ? p.k_scale[b * p.Hkv + hk] * kFp8Bias : 1.f;
-    const float sl = p.scale_log2 * k_mul;  // score -> log2 units
-    // Last key row packed row r sees: pos_first + (r >> gshift) under the
-    // causal mask (-1 for padding rows).
-    auto last_key = [&](int r) {
+    const float sl = p.scale_log2 * k_mul;    // score -> log2 units
+    // Last key row packed row c0 + c sees: pos_first + ((c0 + c) >> gshift)
+    // under the causal mask (-1 for padding rows).
+    auto last_key = [&](int c) {
+      const int r = c0 + c;
       return r < nrows ? (p.causal ? pos_first + (r >> p.gshift) : 0x7FFFFFFF) : -1;
     };
-    float m2[NR], lsum[NR];
+    float m2[CH], lsum[CH];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      m2[r] = -INFINITY;
-      lsum[r] = 0.f;
+    for (int c = 0; c < CH; ++c) {
+      m2[c] = -INFINITY;
+      lsum[c] = 0.f;
     }
     KvCursor<false> cur;
     cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
@@ -339,66 +386,78 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
     bool ok = true;
     while (cur.valid()) {
       const int bsel = (int)(j & 1);
-      if (!(ok = mbar_wait(BAR_S(bsel), (j >> 1) & 1u, abort_flag))) break;
+      if (!(ok = mbar_wait_idle(BAR_S(bsel), (j >> 1) & 1u, abort_flag))) break;
       tc_fence_after();
-      float x[NR];
-      tmem_ld_nr<NR>(T_S(bsel) + lb, x);
+      float x[CH];
+      tmem_ld_ch<CH>(T_S(bsel) + lb + c0, x);
       tc_wait_ld();
-      const int key = cur.k0 + row;
-      const bool kvalid = key < cur.kend;
+      // Masking only where some key is past a row's position or beyond the
+      // chunk's end.  Padding rows need none: their Q rows are zero-filled
+      // and their P^T columns only feed O^T columns that are never written.
+      const bool masked = (cur.kend - cur.k0 < kTileN) || (p.causal && cur.kend - 1 > pos_first);
+      if (masked) {
+        const int key = cur.k0 + row;
+        const bool kvalid = key < cur.kend;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) x[r] = (kvalid && key <= last_key(r)) ? x[r] * sl : -INFINITY;
-      // Column maxima over the tile's 128 keys: each warp, then the four.
+        for (int c = 0; c < CH; ++c) x[c] = (kvalid && key <= last_key(c)) ? x[c] * sl : -INFINITY;
+      } else {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) x[c] *= sl;
+      }
+      // Column maxima over the tile's 128 keys: each warp, then the four lane
+      // quarters ([column][quarter] in shared memory).
       float* rb = red + bsel * 4 * NR;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const int m = __reduce_max_sync(0xFFFFFFFFu, f2ord(x[r]));
-        if (lane == 0) rb[quad * NR + r] = ord2f(m);
+      for (int c = 0; c < CH; ++c) {
+        const int m = __reduce_max_sync(0xFFFFFFFFu, f2ord(x[c]));
+        if (lane == 0) rb[(c0 + c) * 4 + quad] = ord2f(m);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_RED(bsel));
-      if (!(ok = mbar_wait(BAR_RED(bsel), (j >> 1) & 1u, abort_flag))) break;
+      if (!(ok = mbar_wait_idle(BAR_RED(bsel), (j >> 1) & 1u, abort_flag))) break;
       // The base of each row's exponentials trails its running max by at most
       // kRescaleSlack; O^T and the partial sums follow a base that moves.
       bool grow = false;
-      float alpha[NR];
+      float alpha[CH];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const float tm = fmaxf(fmaxf(rb[r], rb[NR + r]), fmaxf(rb[2 * NR + r], rb[3 * NR + r]));
-        alpha[r] = 1.f;
-        if (tm > m2[r] + kRescaleSlack) {
-          alpha[r] = ex2(m2[r] - tm);  // 0 while the row had no key
-          m2[r] = tm;
+      for (int c = 0; c < CH; ++c) {
+        const float4 q4 = *reinterpret_cast<const float4*>(rb + (c0 + c) * 4);
+        const float tm = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
+        alpha[c] = 1.f;
+        if (tm > m2[c] + kRescaleSlack) {
+          alpha[c] = ex2(m2[c] - tm);  // 0 while the row had no key
+          m2[c] = tm;
           grow = true;
         }
       }
       if (grow) {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) lsum[r] *= alpha[r];
+        for (int c = 0; c < CH; ++c) lsum[c] *= alpha[c];
         if (j > 0) {
-          // O^T holds earlier tiles: once the last PV has landed, rescale it
-          // in place (this thread's lane = channel row of O^T).
-          if (!(ok = mbar_wait(BAR_PV((j - 1) & 1), ((j - 1) >> 1) & 1u, abort_flag))) break;
+          // O^T holds earlier tiles: once the last PV has landed, rescale this
+          // warp's columns of its lanes (channels) in place.
+          if (!(ok = mbar_wait_idle(BAR_PV((j - 1) & 1), ((j - 1) >> 1) & 1u, abort_flag))) break;
           tc_fence_after();
-          float o[NR];
-          tmem_ld_nr<NR>(T_O + lb, o);
+          float o[CH];
+          tmem_ld_ch<CH>(T_O + lb + c0, o);
           tc_wait_ld();
 #pragma unroll
-          for (int r = 0; r < NR; ++r) o[r] *= alpha[r];
-          tmem_st_nr<NR>(T_O + lb, o);
+          for (int c = 0; c < CH; ++c) o[c] *= alpha[c];
+          tmem_st_ch<CH>(T_O + lb + c0, o);
           tc_wait_st();
         }
       }
       // P^T as bf16 into buffer bsel (last read by PV_{j-2}), 128-byte
       // swizzled K-major: query row r, key `row` at row r * 128 bytes of the
       // key's 64-key half, 16-byte chunk (key / 8) ^ (r mod 8).
-      if (j >= 2 && !(ok = mbar_wait(BAR_PV(bsel), ((j - 2) >> 1) & 1u, abort_flag))) break;
+      if (j >= 2 && !(ok = mbar_wait_idle(BAR_PV(bsel), ((j - 2) >> 1) & 1u, abort_flag))) break;
       uint8_t* half = smem + L::kPOff + bsel * L::kPBytes + (row >> 6) * (NR * 128);
       const int kh = row & 63;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const float pe = ex2(x[r] - (m2[r] == -INFINITY ? 0.f : m2[r]));
-        lsum[r] += pe;
+      for (int c = 0; c < CH; ++c) {
+        const int r = c0 + c;
+        const float pe = ex2(x[c] - (m2[c] == -INFINITY ? 0.f : m2[c]));
+        lsum[c] += pe;
         *reinterpret_cast<__nv_bfloat16*>(half + r * 128 + (((kh >> 3) ^ (r & 7)) << 4) + (kh & 7) * 2) =
             __float2bfloat16_rn(pe);
       }
@@ -410,41 +469,43 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
       cur.next();
     }
     // ------------------------------ epilogue ------------------------------
-    if (ok) ok = mbar_wait(BAR_DONE, 0, abort_flag);
+    if (ok) ok = mbar_wait_idle(BAR_DONE, 0, abort_flag);
     float* rs = red + 2 * 4 * NR;
     if (ok) {
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        float v = lsum[r];
+      for (int c = 0; c < CH; ++c) {
+        float v = lsum[c];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-        if (lane == 0) rs[quad * NR + r] = v;
+        if (lane == 0) rs[(c0 + c) * 4 + quad] = v;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_SUM);
-      ok = mbar_wait(BAR_SUM, 0, abort_flag);
+      ok = mbar_wait_idle(BAR_SUM, 0, abort_flag);
     }
     if (ok) {
       tc_fence_after();
-      float o[NR];
+      float o[CH];
       if (j > 0) {
-        tmem_ld_nr<NR>(T_O + lb, o);
+        tmem_ld_ch<CH>(T_O + lb + c0, o);
         tc_wait_ld();
       } else {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) o[r] = 0.f;
+        for (int c = 0; c < CH; ++c) o[c] = 0.f;
       }
       const float v_mul = kKV8 ? p.v_scale[b * p.Hkv + hk] : 1.f;
       const int dch = row;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int c = 0; c < CH; ++c) {
+        const int r = c0 + c;
         if (r >= nrows) continue;
-        const float l = rs[r] + rs[NR + r] + rs[2 * NR + r] + rs[3 * NR + r];
+        const float4 s4 = *reinterpret_cast<const float4*>(rs + r * 4);
+        const float l = (s4.x + s4.y) + (s4.z + s4.w);
         const float inv = l > 0.f ? v_mul / l : 0.f;
-        const float val = (kKV8 ? o[r] * kFp8Bias : o[r]) * inv;
-        const long long t = tok0 + r / p.G;
-        const int h = hk * p.G + r % p.G;
-        const float lse_v = l > 0.f ? (m2[r] + log2f(l)) * kLn2 : -INFINITY;
+        const float val = (kKV8 ? o[c] * kFp8Bias : o[c]) * inv;
+        const long long t = tok0 + (r >> p.gshift);
+        const int h = hk * p.G + (r & (p.G - 1));
+        const float lse_v = l > 0.f ? (m2[c] + log2f(l)) * kLn2 : -INFINITY;
         if (MODE == kModeSplit) {
           p.o_part[(((long long)(sigma * p.B + b) * p.N_q + t) * p.Hq + h) * kDecD + dch] = val;
           if (row == 0) p.lse_part[((long long)(sigma * p.B + b) * p.Hq + h) * p.N_q + t] = lse_v;
@@ -455,11 +516,10 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
         }
       }
     }
-  } else if (kKV8 && warp >= 8) {
+  } else if (kKV8 && warp >= 12) {
     // ============================ FP8 converters ============================
     if constexpr (kKV8) {
-      reg_dealloc<96>();
-      const int ct = (int)threadIdx.x - 256;
+      const int ct = (int)threadIdx.x - 384;
       KvCursor<false> cur;
       cur.init((int)p.chunk, lim, p.P, home, s_begin, s_end);
       uint32_t f = 0;
@@ -467,8 +527,8 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 384 : 256, 1) decode_sm100_kernel
       while (ok && cur.valid()) {
         for (int kv = 0; kv < 2; ++kv) {
           const uint32_t slot8 = f % NSLOT8, slot = f % NSLOT;
-          if (!(ok = mbar_wait(BAR_F8_FULL(slot8), (f / NSLOT8) & 1u, abort_flag))) break;
-          if (!(ok = mbar_wait(BAR_KV_EMPTY(slot), ((f / NSLOT) & 1u) ^ 1u, abort_flag))) break;
+          if (!(ok = mbar_wait_idle(BAR_F8_FULL(slot8), (f / NSLOT8) & 1u, abort_flag))) break;
+          if (!(ok = mbar_wait_idle(BAR_KV_EMPTY(slot), ((f / NSLOT) & 1u) ^ 1u, abort_flag))) break;
           convert_fp8_tile<kDecD>(smem + L::kF8Off + slot8 * L::kF8Bytes, smem + L::kKVOff + slot * L::kTileBytes,
                                   ct);
           fence_proxy_async_smem();
@@ -496,17 +556,6 @@ cudaError_t launch_dec_cfg(const DecParams& prm, long long grid, cudaStream_t st
   using L = DecLayout<NR, NSLOT, NSLOT8>;
   static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
   auto kern = decode_sm100_kernel<NR, NSLOT, MODE, NSLOT8>;
-  if constexpr (NSLOT8 > 0) {
-    // The in-kernel register split assumes 168 registers per thread.
-    static int regs = -1;
-    if (regs < 0) {
-      cudaFuncAttributes fa;
-      cudaError_t e0 = cudaFuncGetAttributes(&fa, kern);
-      if (e0 != cudaSuccess) return e0;
-      regs = fa.numRegs;
-    }
-    if (regs != 168) return cudaErrorInvalidConfiguration;
-  }
   static unsigned long long attr_set_mask = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -517,7 +566,7 @@ cudaError_t launch_dec_cfg(const DecParams& prm, long long grid, cudaStream_t st
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&attr_set_mask, bit, __ATOMIC_RELEASE);
   }
-  kern<<<(unsigned)grid, NSLOT8 > 0 ? 384 : 256, L::kAlloc, st>>>(prm);
+  kern<<<(unsigned)grid, NSLOT8 > 0 ? 512 : 384, L::kAlloc, st>>>(prm);
   return count_launch(cudaGetLastError());
 }
 
@@ -598,13 +647,14 @@ cudaError_t launch_decode_sm100(const ProblemArgs& a, int mode, cudaStream_t st)
   }
   const long long grid = (long long)a.B * a.Hkv * prm.n_qblk * prm.S;
   if (a.kv8) {
-    if (NR == 16) return mode == kModeSplit ? launch_dec_cfg<16, 4, kModeSplit, 4>(prm, grid, st)
-                                            : launch_dec_cfg<16, 4, kModeFinal, 4>(prm, grid, st);
+    if (NR == 16)
+      return mode == kModeSplit ? launch_dec_cfg<16, RA_DEC8_NSLOT, kModeSplit, RA_DEC8_NSLOT8>(prm, grid, st)
+                                : launch_dec_cfg<16, RA_DEC8_NSLOT, kModeFinal, RA_DEC8_NSLOT8>(prm, grid, st);
     return mode == kModeSplit ? launch_dec_cfg<32, 4, kModeSplit, 4>(prm, grid, st)
                               : launch_dec_cfg<32, 4, kModeFinal, 4>(prm, grid, st);
   }
-  if (NR == 16) return mode == kModeSplit ? launch_dec_cfg<16, 6, kModeSplit, 0>(prm, grid, st)
-                                          : launch_dec_cfg<16, 6, kModeFinal, 0>(prm, grid, st);
+  if (NR == 16) return mode == kModeSplit ? launch_dec_cfg<16, RA_DEC_NSLOT, kModeSplit, 0>(prm, grid, st)
+                                          : launch_dec_cfg<16, RA_DEC_NSLOT, kModeFinal, 0>(prm, grid, st);
   return mode == kModeSplit ? launch_dec_cfg<32, 6, kModeSplit, 0>(prm, grid, st)
                             : launch_dec_cfg<32, 6, kModeFinal, 0>(prm, grid, st);
 }

@@ -333,51 +333,72 @@ __device__ __forceinline__ void warp_arrive_after_tc(uint32_t bar, int lane) {
 }
 
 // Four E4M3 codes (bytes of w, lowest address first) to two bf16x2 words
-// holding each code's value times 2^-120 (kFp8Bias), with integer byte moves
+// holding each code's value times 2^-120 (kFp8Bias), with integer operations
 // only.  An E4M3 code s.eeee.mmm placed in a bf16 word as s.0000eeee.mmm0000
 // reads as 2^(e-127) (1 + m/8) = 2^-120 * 2^(e-7) (1 + m/8) for e >= 1, and
 // as the subnormal 2^-126 * m/8 = 2^-120 * 2^-6 * m/8 for e = 0: exact for
 // every finite code.  The 2^120 goes back in through the scales.
 constexpr float kFp8Bias = 1.329227995784916e36f;  // 2^120
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
+  // Two codes into the low bytes of the two 16-bit halves: 0000 0000 seee emmm.
+  const uint32_t x = __byte_perm(w, 0, sel);
+  // Moving the sign from bit 7 to bit 15 while the code moves up 4 bits:
+  // 16 * (x + 15 * sign) = (code << 4) - (sign << 4) + (sign << 8), as two
+  // multiply-adds (FMA pipe) and one mask (ALU pipe).
+  const uint32_t sgn = x & 0x00800080u;
+  return __umul24(sgn, 15u) * 16u + x * 16u;
+}
 __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t em = w & 0x7F7F7F7Fu;  // exponent and mantissa of each code
-  const uint32_t sg = w & 0x80808080u;  // sign of each code
-  // Codes 0, 1 -> bf16 halves of lo; codes 2, 3 -> halves of hi.  Exponent
-  // and mantissa land in the low byte of each half and move up 4 bits; the
-  // sign byte lands in the high byte (bit 7 -> bit 15).
-  lo = __byte_perm(em, 0, 0x4140) * 16u + __byte_perm(sg, 0, 0x1404);
-  hi = __byte_perm(em, 0, 0x4342) * 16u + __byte_perm(sg, 0, 0x3424);
+  lo = e4m3x2_to_bf16x2(w, 0x4140);  // codes 0, 1
+  hi = e4m3x2_to_bf16x2(w, 0x4342);  // codes 2, 3
 }
 
-// Decode one FP8 tile (128 keys x D codes, row-major, as the TMA copy left it)
-// into a bf16 tile in the layout a TMA copy with 128-byte swizzle produces:
-// 64-element column blocks of 128 rows x 128 bytes, the 16-byte chunk j of
-// row r stored at chunk j ^ (r mod 8).  Thread ct of the converter warpgroup
-// takes every 128th 16-code chunk; a warp reads 512 contiguous bytes.
+// Decode one FP8 tile (128 keys x D codes) into a bf16 tile in the layout a
+// TMA copy with 128-byte swizzle produces: 64-element column blocks of
+// 128 rows x 128 bytes, the 16-byte chunk j of row r stored at j ^ (r mod 8).
+// Thread ct of the converter warpgroup converts 16-code chunks.
+//
+// d = 128: the FP8 tile also arrives 128-byte swizzled (its 16-code chunk c
+// of row r at c ^ (r mod 8)).  Eight consecutive threads (one shared-memory
+// phase of a 16-byte access) take the same chunk column of eight
+// consecutive rows, so their loads and their stores fall on eight distinct
+// bank groups.  d = 64: row-major codes, threads along the row.
+// Every chunk of a thread has the same column and the same row mod 8, so all
+// its addresses are one base plus constants.
 template <int D>
 __device__ __forceinline__ void convert_fp8_tile(const uint8_t* src, uint8_t* dst, int ct) {
   constexpr int kChunksPerRow = D / 16;
   constexpr int kPerThread = kTileN * kChunksPerRow / 128;
+  int r0, cc, row_step, src_chunk;
+  if constexpr (D == 128) {
+    const int a = ct >> 3, b = ct & 7;
+    cc = a & 7;
+    r0 = b + 8 * (a >> 3);  // rows r0 + 16 i
+    row_step = 16;
+    src_chunk = cc ^ b;     // swizzled position of chunk cc in row r0 (r0 mod 8 = b)
+  } else {
+    r0 = ct / kChunksPerRow;
+    cc = ct % kChunksPerRow;
+    row_step = 128 / kChunksPerRow;
+    src_chunk = cc;
+  }
+  const uint8_t* s0 = src + r0 * D + src_chunk * 16;
+  const int j0 = (cc % 4) * 2;  // 16 codes = 32 bytes of bf16: chunks j0, j0 + 1
+  uint8_t* d0 = dst + (cc / 4) * (kTileN * 128) + r0 * 128;
+  const int a0 = (j0 ^ (r0 & 7)) << 4, a1 = ((j0 + 1) ^ (r0 & 7)) << 4;
   // All of this thread's loads first, so their latencies overlap.
   uint4 w[kPerThread];
 #pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
-    const int c = ct + 128 * i;
-    w[i] = *reinterpret_cast<const uint4*>(src + (c / kChunksPerRow) * D + (c % kChunksPerRow) * 16);
-  }
+  for (int i = 0; i < kPerThread; ++i) w[i] = *reinterpret_cast<const uint4*>(s0 + i * row_step * D);
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
-    const int c = ct + 128 * i;
-    const int r = c / kChunksPerRow, cc = c % kChunksPerRow;
     uint4 o0, o1;
     e4m3x4_to_bf16x4(w[i].x, o0.x, o0.y);
     e4m3x4_to_bf16x4(w[i].y, o0.z, o0.w);
     e4m3x4_to_bf16x4(w[i].z, o1.x, o1.y);
     e4m3x4_to_bf16x4(w[i].w, o1.z, o1.w);
-    const int j0 = (cc % 4) * 2;  // 16 codes = 32 bytes of bf16: chunks j0, j0 + 1
-    uint8_t* row = dst + (cc / 4) * (kTileN * 128) + r * 128;
-    *reinterpret_cast<uint4*>(row + ((j0 ^ (r & 7)) << 4)) = o0;
-    *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (r & 7)) << 4)) = o1;
+    *reinterpret_cast<uint4*>(d0 + i * row_step * 128 + a0) = o0;
+    *reinterpret_cast<uint4*>(d0 + i * row_step * 128 + a1) = o1;
   }
 }
 
@@ -1026,8 +1047,9 @@ cudaError_t launch_cfg(const Sm100Params& prm, long long grid, cudaStream_t st) 
   return count_launch(cudaGetLastError());
 }
 
-// FP8 codes, one row of d bytes per (token, head): 128-key boxes without
-// swizzle (the converters re-lay them out).
+// FP8 codes, one row of d bytes per (token, head): 128-key boxes, 128-byte
+// swizzled at d = 128 (the converters read them conflict-free), plain at
+// d = 64.
 CUresult encode_map_u8(CUtensorMap* m, const void* base, int d, int H, long long N, int B) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return CUDA_ERROR_NOT_FOUND;
@@ -1036,8 +1058,8 @@ CUresult encode_map_u8(CUtensorMap* m, const void* base, int d, int H, long long
   cuuint32_t box[4] = {(cuuint32_t)d, 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+             CU_TENSOR_MAP_INTERLEAVE_NONE, d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 CUresult encode_map(CUtensorMap* m, const void* base, int d, int H, long long N, int B, int box_heads = 1) {
