@@ -42,13 +42,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.830734 GB read + 0.255677 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.086411e9, "src": "d6d6b77a5bb63a09"},
-    # profiles/fwd_sm100_decode_Nq1_Nkv65536.md: 1.073881 GB read + 0.007975 GB written.
-    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.081856e9, "src": "2e7ad4d545362cff"},
-    # The full-length decode scales the quarter-length capture by its 4x KV
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.829857 GB read + 0.254630 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.084487e9, "src": "67b60eea843784ec"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073909 GB read + 0.004924 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078833e9, "src": "67b60eea843784ec"},
+    # The full-length decodes scale the quarter-length captures by their 4x KV
     # length (traffic is K/V streaming, proportional to N_kv).
-    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.081856e9, "src": "2e7ad4d545362cff"},
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078833e9, "src": "67b60eea843784ec"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537088 GB read + 0.004268 GB written.
+    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541356e9, "src": "67b60eea843784ec"},
+    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541356e9, "src": "67b60eea843784ec"},
 }
 
 
@@ -94,6 +97,19 @@ def flops_of(w: workloads.Workload) -> float:
     else:
         pairs = float(w.N_q * w.N_kv)
     return 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def kernel_name(w: workloads.Workload, bwd: bool) -> str:
+    """The dominant kernel of a step (the library's routing rule for d = 128
+    incremental queries with at most 16 packed rows per KV head)."""
+    if bwd:
+        return "bwd_prep + bwd_dkdv + bwd_dq (whole step)"
+    if w.dtype != "bf16":
+        return "simt_attn_kernel"
+    fp8 = " (FP8 KV, converter warpgroup)" if w.kv_dtype == "fp8" else ""
+    if w.d == 128 and w.cache_idx > 0 and w.window < 0 and (w.Hq // w.Hkv) * w.N_q <= 16:
+        return "decode_sm100_kernel" + fp8
+    return "fwd_sm100_kernel" + fp8
 
 
 def window_anchor_pairs(n: int, window: int, period: int) -> float:
@@ -555,9 +571,7 @@ def main():
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} ({peak_kind if bound == 'tensor' else bound})",
-                     "kernel": ("bwd_prep + bwd_dkdv + bwd_dq (whole step)" if bwd else
-                                "fwd_sm100_kernel (FP8 KV, converter warpgroup)" if w.kv_dtype == "fp8" else
-                                "fwd_sm100_kernel" if w.dtype == "bf16" else "simt_attn_kernel"),
+                     "kernel": kernel_name(w, bwd),
                      "algorithmic_per_launch": flops if unit == "TFLOP/s" else hbm_bytes_of(w)},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
