@@ -103,6 +103,16 @@ constexpr int kDecD = 128;  // channels (the decode kernel serves d = 128)
 #ifndef RA_DEC_HEADS_INNER
 #define RA_DEC_HEADS_INNER 1
 #endif
+// Warps whose row columns are all padding skip their arithmetic (1, measured
+// faster: they leave issue slots to the others) or not (0).
+#ifndef RA_DEC_IDLE_PAD
+#define RA_DEC_IDLE_PAD 1
+#endif
+// Column maxima by shuffle trees (1, measured faster) or integer warp
+// reductions (0).
+#ifndef RA_DEC_SHFL_MAX
+#define RA_DEC_SHFL_MAX 1
+#endif
 // CTAs per SM the decode kernel is compiled for.
 #ifndef RA_DEC_MINB
 #define RA_DEC_MINB 1
@@ -389,6 +399,14 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 512 : 384, RA_DEC_MINB) decode_sm
       if (!(ok = mbar_wait_idle(BAR_S(bsel), (j >> 1) & 1u, abort_flag))) break;
       tc_fence_after();
       float x[CH];
+#if RA_DEC_IDLE_PAD
+      // A warp whose row columns are all padding only keeps pace on the
+      // barriers (its P^T columns feed O^T columns that are never written).
+      const bool pad_only = c0 >= nrows;
+#else
+      const bool pad_only = false;
+#endif
+      if (!pad_only) {
       tmem_ld_ch<CH>(T_S(bsel) + lb + c0, x);
       tc_wait_ld();
       // Masking only where some key is past a row's position or beyond the
@@ -404,17 +422,37 @@ __global__ void __launch_bounds__(NSLOT8 > 0 ? 512 : 384, RA_DEC_MINB) decode_sm
 #pragma unroll
         for (int c = 0; c < CH; ++c) x[c] *= sl;
       }
+      }
       // Column maxima over the tile's 128 keys: each warp, then the four lane
       // quarters ([column][quarter] in shared memory).
       float* rb = red + bsel * 4 * NR;
+      if (!pad_only) {
+#if RA_DEC_SHFL_MAX
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        float m = x[c];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) rb[(c0 + c) * 4 + quad] = m;
+      }
+#else
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
         const int m = __reduce_max_sync(0xFFFFFFFFu, f2ord(x[c]));
         if (lane == 0) rb[(c0 + c) * 4 + quad] = ord2f(m);
       }
+#endif
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_RED(bsel));
       if (!(ok = mbar_wait_idle(BAR_RED(bsel), (j >> 1) & 1u, abort_flag))) break;
+      if (pad_only) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR_P(bsel));
+        ++j;
+        cur.next();
+        continue;
+      }
       // The base of each row's exponentials trails its running max by at most
       // kRescaleSlack; O^T and the partial sums follow a base that moves.
       bool grow = false;
