@@ -43,15 +43,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
     # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.829857 GB read + 0.254630 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.084487e9, "src": "67b60eea843784ec"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073909 GB read + 0.004924 GB written.
-    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078833e9, "src": "67b60eea843784ec"},
+    "llama7b_prefill_N32768": {"bytes": 1.084487e9, "src": "25f212287f8997c7"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073930 GB read + 0.004202 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078132e9, "src": "7ee2ab864cd3d8e7"},
     # The full-length decodes scale the quarter-length captures by their 4x KV
     # length (traffic is K/V streaming, proportional to N_kv).
-    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078833e9, "src": "67b60eea843784ec"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537088 GB read + 0.004268 GB written.
-    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541356e9, "src": "67b60eea843784ec"},
-    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541356e9, "src": "67b60eea843784ec"},
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078132e9, "src": "7ee2ab864cd3d8e7"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537044 GB read + 0.004457 GB written.
+    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541501e9, "src": "7ee2ab864cd3d8e7"},
+    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541501e9, "src": "7ee2ab864cd3d8e7"},
     # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step (prep + dK/dV + dQ):
     # 0.541 + 0.011, 1.087 + 0.509, 1.084 + 0.255 GB read + written.
     "llama7b_prefill_N32768 bwd": {"bytes": 3.487206e9, "src": "e66ff11ce68aa9f4"},
@@ -59,7 +59,12 @@ NCU_TRAFFIC = {
 
 
 # Sources that do not affect a pass's kernels, left out of its hash.
-_NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh"}, "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh"}}
+# The kernel families: "fwd" (the general forward), "decode" (the keys-on-M
+# decode kernel, which shares the FP8 converter and cursor code of the
+# forward's sources) and "bwd".
+_NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh", "decode_sm100.cuh"},
+                "decode": {"bwd_sm100.cuh", "fwd_simt.cuh"},
+                "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh"}}
 
 
 def kernel_source_hash(pass_: str = "fwd") -> str:
@@ -549,7 +554,7 @@ def main():
         bound, unit = "hbm", "GB/s"
         achieved = hbm_bytes_of(w) / (launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
-    src_hash = kernel_source_hash(args.pass_)
+    src_hash = kernel_source_hash("bwd" if bwd else ("decode" if kernel_name(w, bwd).startswith("decode") else "fwd"))
     tr = NCU_TRAFFIC.get(w.name + (" bwd" if bwd else ""))
     traffic = tr["bytes"] if tr and tr.get("src") == src_hash else None
     cpu = None
