@@ -425,13 +425,18 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
 // ---------------------------------------------------------------- dQ
 template <int D>
 struct DqLayout {
+  // K_j is read by S_j and, last, by dQ_j; V_j only by dP_j.  Three K slots
+  // let K_{j+1} load while dQ_{j-1} still holds its slot (two stages put a
+  // whole load latency in front of S_{j+1}); V needs two.
+  static constexpr int kKSlots = 3, kVSlots = 2;
   static constexpr int kTile = kBT * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kDo = kQ + kTile;
-  static constexpr int kStage0 = kDo + kTile;  // per stage: K, V
-  static constexpr int kStageBytes = 2 * kTile;
-  static constexpr int kBars = kStage0 + 2 * kStageBytes;  // q_full, kf[2], ke[2], s[2], ds, done, drain, dp
-  static constexpr int kMisc = kBars + 12 * 8;
+  static constexpr int kK0 = kDo + kTile;
+  static constexpr int kV0 = kK0 + kKSlots * kTile;
+  // q_full, kf[3], ke[3], vf[2], ve[2], s[2], ds, done, drain, dp
+  static constexpr int kBars = kV0 + kVSlots * kTile;
+  static constexpr int kMisc = kBars + 17 * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024 < 120 * 1024 ? 120 * 1024 : kBytes + 1024;
 };
@@ -444,14 +449,17 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBars;
   const uint32_t BAR_Q = bar0;
-  auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto BAR_KE = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto BAR_S = [&](int s) { return bar0 + 8u * (5 + s); };
-  const uint32_t BAR_DS = bar0 + 8u * 7, BAR_DONE = bar0 + 8u * 8, BAR_DRAIN = bar0 + 8u * 9, BAR_DP = bar0 + 8u * 10;
+  auto BAR_KF = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto BAR_KE = [&](int i) { return bar0 + 8u * (4 + i); };
+  auto BAR_VF = [&](int i) { return bar0 + 8u * (7 + i); };
+  auto BAR_VE = [&](int i) { return bar0 + 8u * (9 + i); };
+  auto BAR_S = [&](int s) { return bar0 + 8u * (11 + s); };
+  const uint32_t BAR_DS = bar0 + 8u * 13, BAR_DONE = bar0 + 8u * 14, BAR_DRAIN = bar0 + 8u * 15, BAR_DP = bar0 + 8u * 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  auto stage_k = [&](int s) { return sbase + L::kStage0 + s * L::kStageBytes; };
-  auto stage_v = [&](int s) { return stage_k(s) + L::kTile; };
+  constexpr int KS = L::kKSlots, VS = L::kVSlots;
+  auto slot_k = [&](int j) { return sbase + L::kK0 + (j % KS) * L::kTile; };  // K_j
+  auto slot_v = [&](int j) { return sbase + L::kV0 + (j % VS) * L::kTile; };  // V_j
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Head-major order (the resident CTAs share one KV head's K / V in L2),
@@ -472,11 +480,15 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR_KF(s), 1);
-      mbar_init(BAR_KE(s), 1);
-      mbar_init(BAR_S(s), 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(BAR_KF(i), 1);
+      mbar_init(BAR_KE(i), 1);
     }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(BAR_VF(i), 1);
+      mbar_init(BAR_VE(i), 1);
+    }
+    for (int s = 0; s < 2; ++s) mbar_init(BAR_S(s), 1);
     mbar_init(BAR_DS, 4);
     mbar_init(BAR_DONE, 1);
     mbar_init(BAR_DRAIN, 1);
@@ -506,15 +518,18 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
       tma_tile(sbase + L::kQ, &p.tm_q, BAR_Q, D, h, t0, b);
       tma_tile(sbase + L::kDo, &p.tm_do, BAR_Q, D, h, t0, b);
       for (int j = 0; j < n_jt; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(BAR_KE(s), ((j >> 1) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(BAR_KF(s), 2 * L::kTile);
-        tma_tile(stage_k(s), &p.tm_k, BAR_KF(s), D, hk, j * kBT, b);
-        tma_tile(stage_v(s), &p.tm_v, BAR_KF(s), D, hk, j * kBT, b);
+        if (!mbar_wait(BAR_KE(j % KS), ((j / KS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR_KF(j % KS), L::kTile);
+        tma_tile(slot_k(j), &p.tm_k, BAR_KF(j % KS), D, hk, j * kBT, b);
+        if (!mbar_wait(BAR_VE(j % VS), ((j / VS) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR_VF(j % VS), L::kTile);
+        tma_tile(slot_v(j), &p.tm_v, BAR_VF(j % VS), D, hk, j * kBT, b);
       }
+      // Let in-flight copies land before the CTA can exit.
       volatile int no_abort = 0;
       mbar_wait(BAR_Q, 0, &no_abort);
-      for (int j = n_jt > 2 ? n_jt - 2 : 0; j < n_jt; ++j) mbar_wait(BAR_KF(j & 1), (j >> 1) & 1, &no_abort);
+      for (int j = n_jt > KS ? n_jt - KS : 0; j < n_jt; ++j) mbar_wait(BAR_KF(j % KS), (j / KS) & 1, &no_abort);
+      for (int j = n_jt > VS ? n_jt - VS : 0; j < n_jt; ++j) mbar_wait(BAR_VF(j % VS), (j / VS) & 1, &no_abort);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -528,29 +543,37 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
       // two phases ahead of the elementwise warps.
       bool ok = mbar_wait(BAR_Q, 0, abort_flag);
       tc_fence_after();
+      auto issue_dp = [&](int j) {  // dP_j = dout V_j^T, then V_j's slot is free
+        mma_rows_x_rows<D>(T_DP, sbase + L::kDo, slot_v(j));
+        tc_commit(BAR_DP);
+        tc_commit(BAR_VE(j % VS));
+      };
       if (ok && n_jt > 0 && (ok = mbar_wait(BAR_KF(0), 0, abort_flag))) {
         tc_fence_after();
-        mma_rows_x_rows<D>(T_S(0), sbase + L::kQ, stage_k(0));   // S = Q K^T
+        mma_rows_x_rows<D>(T_S(0), sbase + L::kQ, slot_k(0));   // S = Q K^T
         tc_commit(BAR_S(0));
-        mma_rows_x_rows<D>(T_DP, sbase + L::kDo, stage_v(0));    // dP = dout V^T
-        tc_commit(BAR_DP);
+        if ((ok = mbar_wait(BAR_VF(0), 0, abort_flag))) {
+          tc_fence_after();
+          issue_dp(0);
+        }
       }
       for (int j = 0; j < n_jt && ok; ++j) {
         const int s = j & 1;
         const bool more = j + 1 < n_jt;
         if (more) {
-          if (!(ok = mbar_wait(BAR_KF(s ^ 1), ((j + 1) >> 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(BAR_KF((j + 1) % KS), ((j + 1) / KS) & 1, abort_flag))) break;
           tc_fence_after();
-          mma_rows_x_rows<D>(T_S(s ^ 1), sbase + L::kQ, stage_k(s ^ 1));
+          mma_rows_x_rows<D>(T_S(s ^ 1), sbase + L::kQ, slot_k(j + 1));
           tc_commit(BAR_S(s ^ 1));
         }
         if (!(ok = mbar_wait(BAR_DS, j & 1, abort_flag))) break;
         tc_fence_after();
-        mma_tmem_x_tile<D>(T_DQ, T_S(s), stage_k(s), j > 0);    // dQ += dS K
-        tc_commit(BAR_KE(s));
+        mma_tmem_x_tile<D>(T_DQ, T_S(s), slot_k(j), j > 0);    // dQ += dS K
+        tc_commit(BAR_KE(j % KS));
         if (more) {
-          mma_rows_x_rows<D>(T_DP, sbase + L::kDo, stage_v(s ^ 1));
-          tc_commit(BAR_DP);
+          if (!(ok = mbar_wait(BAR_VF((j + 1) % VS), ((j + 1) / VS) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_dp(j + 1);
         }
       }
       tc_commit(BAR_DONE);
