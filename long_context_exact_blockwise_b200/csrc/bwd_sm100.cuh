@@ -22,8 +22,11 @@
 //                     over KV tiles; S = Q K^T, dP = dout V^T, dS, then
 //                     dQ += dS K in TMEM.
 // Warp roles in both: warp 0 TMA, warp 1 MMA issue (one thread), warp 2
-// TMEM allocation, warps 4..7 the elementwise warpgroup (thread = TMEM
-// lane = tile row).  Every mbarrier wait is bounded as in the forward.
+// TMEM allocation, warps 4.. the elementwise warps.  An elementwise thread
+// owns one TMEM lane (tile row) and one column group: two warps share each
+// lane quarter, one per half of the tile's 128 columns, so two warps per SM
+// sub-partition overlap their exponential chains.  Every mbarrier wait is
+// bounded as in the forward.
 #pragma once
 
 #include <cstdlib>
@@ -37,6 +40,31 @@ namespace ra {
 namespace {
 
 constexpr int kBT = 128;  // tile rows (queries or keys)
+
+// Elementwise warps of each kernel: 4 (one per TMEM lane quarter) or 8 (two
+// per quarter, one per column half).
+#ifndef RA_BWD_EW_DKDV
+#define RA_BWD_EW_DKDV 8
+#endif
+#ifndef RA_BWD_EW_DQ
+#define RA_BWD_EW_DQ 4
+#endif
+
+template <int EW>
+struct EwSplit {
+  static_assert(EW == 4 || EW == 8, "elementwise warps: one or two per TMEM lane quarter");
+  static constexpr int kNH = EW / 4;        // column groups per tile row
+  static constexpr int kCW = kBT / kNH;     // columns per group
+  static constexpr int kThreads = 128 + 32 * EW;
+  // A column group g writes its bf16 pairs (16 columns per 32 values) over
+  // the start of its own fp32 columns [g kCW, (g+1) kCW), so no group
+  // overwrites values another has yet to read.  TMEM column of the packed
+  // operand's 16 contraction elements kk (as A of an MMA from TMEM):
+  static __device__ __forceinline__ constexpr uint32_t packed_col(int kk) {
+    return (uint32_t)((kk / (kCW / 16)) * kCW + (kk % (kCW / 16)) * 8);
+  }
+};
+constexpr int kEwDkdv = RA_BWD_EW_DKDV, kEwDq = RA_BWD_EW_DQ;
 
 // 1-D bulk copy global -> shared, completion on an mbarrier (16-byte aligned
 // addresses, size a multiple of 16).
@@ -82,14 +110,15 @@ __device__ __forceinline__ void mma_rows_x_rows(uint32_t d_tmem, uint32_t a_addr
   }
 }
 
-// D(tmem, M=128 x N=D) (+)= A(tmem, bf16 128 x 128) B(128 rows x D, MN-major).
-template <int D>
+// D(tmem, M=128 x N=D) (+)= A(tmem, bf16 128 x 128 packed by column group)
+// B(128 rows x D, MN-major).
+template <int D, int EW>
 __device__ __forceinline__ void mma_tmem_x_tile(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(kBT, D, 1);
   const uint64_t bd = mnmajor_desc(b_addr);
 #pragma unroll
   for (int kk = 0; kk < kBT / 16; ++kk)
-    umma_ts(d_tmem, a_tmem + kk * 8, bd + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts(d_tmem, a_tmem + EwSplit<EW>::packed_col(kk), bd + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int D, int head, int row,
@@ -140,8 +169,9 @@ struct DkdvLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using L = DkdvLayout<D>;
+  constexpr int kEw = kEwDkdv, kNH = EwSplit<kEw>::kNH, kCW = EwSplit<kEw>::kCW;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -182,14 +212,14 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     mbar_init(BAR_KV, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR_QF(s), 1);
-      mbar_init(BAR_QE(s), 1 + 4);  // MMA commit + one arrival per elementwise warp
+      mbar_init(BAR_QE(s), 1 + kEw);  // MMA commit + one arrival per elementwise warp
     }
     mbar_init(BAR_S, 1);
-    mbar_init(BAR_P, 4);
+    mbar_init(BAR_P, kEw);
     mbar_init(BAR_DONE, 1);
     mbar_init(BAR_DRAIN, 1);
     mbar_init(BAR_DP, 1);
-    mbar_init(BAR_DS, 4);
+    mbar_init(BAR_DS, kEw);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -260,7 +290,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
         const bool more = w + 1 < n_work;
         if (!(ok = mbar_wait(BAR_P, w & 1, abort_flag))) break;
         tc_fence_after();
-        mma_tmem_x_tile<D>(T_DV, T_ST, stage_do(s), w > 0);   // dV += P^T dout
+        mma_tmem_x_tile<D, kEw>(T_DV, T_ST, stage_do(s), w > 0);   // dV += P^T dout
         if (more) {
           if (!(ok = mbar_wait(BAR_QF(s ^ 1), ((w + 1) >> 1) & 1, abort_flag))) break;
           tc_fence_after();
@@ -269,7 +299,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
         }
         if (!(ok = mbar_wait(BAR_DS, w & 1, abort_flag))) break;
         tc_fence_after();
-        mma_tmem_x_tile<D>(T_DK, T_DPT, stage_q(s), w > 0);   // dK += dS^T Q
+        mma_tmem_x_tile<D, kEw>(T_DK, T_DPT, stage_q(s), w > 0);   // dK += dS^T Q
         tc_commit(BAR_QE(s));
         if (more) {
           mma_rows_x_rows<D>(T_DPT, sbase + L::kV, stage_do(s ^ 1));
@@ -283,8 +313,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     }
   } else if (warp >= 4) {
     const int quad = warp & 3;
+    const int grp = (warp - 4) >> 2;  // query columns [grp kCW, (grp+1) kCW)
+    const int g0 = grp * kCW;
     const int r = quad * 32 + lane;  // key row of the tile
-    const uint32_t lb = (uint32_t)(quad * 32) << 16;
+    const uint32_t lq = (uint32_t)(quad * 32) << 16;
+    const uint32_t lb = lq + (uint32_t)g0;
     const long long key = (long long)j0 + r;
     const float sl = p.scale_log2;
     bool ok = true;
@@ -304,22 +337,22 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
       long long cm = p.causal ? (key + p.k_pos0 - p.q_pos0) - (long long)qt * kBT : -1;
       const int cmin = (int)(cm < 0 ? 0 : (cm > kBT ? kBT : cm));
       // Phase 1: P^T (kept in registers for phase 2), bf16 over S^T.
-      float pv[kBT];
+      float pv[kCW];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float st[32];
-        tmem_ld32(T_ST + lb + c * 32, st);
-        tc_wait_ld();
+      for (int c = 0; c < kCW / 32; ++c) tmem_ld32(T_ST + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
+      tc_wait_ld();
+#pragma unroll
+      for (int c = 0; c < kCW / 32; ++c) {
         uint32_t up[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const int q0 = c * 32 + i;
-          float p0 = ex2(fmaf(st[i], sl, -lse2[q0]));
-          float p1 = ex2(fmaf(st[i + 1], sl, -lse2[q0 + 1]));
+          const int l0 = c * 32 + i, q0 = g0 + l0;
+          float p0 = ex2(fmaf(pv[l0], sl, -lse2[q0]));
+          float p1 = ex2(fmaf(pv[l0 + 1], sl, -lse2[q0 + 1]));
           if (q0 < cmin) p0 = 0.f;
           if (q0 + 1 < cmin) p1 = 0.f;
-          pv[q0] = p0;
-          pv[q0 + 1] = p1;
+          pv[l0] = p0;
+          pv[l0 + 1] = p1;
           up[i / 2] = pack_bf16x2(p0, p1);
         }
         tmem_st16(T_ST + lb + c * 16, up);
@@ -332,15 +365,15 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
       if (!(ok = mbar_wait(BAR_DP, w & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kCW / 32; ++c) {
         float dpt[32];
         tmem_ld32(T_DPT + lb + c * 32, dpt);
         tc_wait_ld();
         uint32_t uds[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const int q0 = c * 32 + i;
-          uds[i / 2] = pack_bf16x2(pv[q0] * (dpt[i] - dD[q0]), pv[q0 + 1] * (dpt[i + 1] - dD[q0 + 1]));
+          const int l0 = c * 32 + i, q0 = g0 + l0;
+          uds[i / 2] = pack_bf16x2(pv[l0] * (dpt[i] - dD[q0]), pv[l0 + 1] * (dpt[i + 1] - dD[q0 + 1]));
         }
         tmem_st16(T_DPT + lb + c * 16, uds);
       }
@@ -357,16 +390,17 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
       tc_fence_after();
       const bool valid = key < p.N_kv;
       const long long off = (((long long)b * p.N_kv + (valid ? key : 0)) * p.Hkv + hk) * D;
+      const int e0 = grp * (D / kNH);  // this warp's dV / dK columns
       if (p.accumulate) {
         // dv += P^T dout, dk += scale dS^T Q into the caller's float32 rows
         // (a key no query of this call sees is left as it was).
-        float* dv = static_cast<float*>(p.dv) + off;
-        float* dk = static_cast<float*>(p.dk) + off;
+        float* dv = static_cast<float*>(p.dv) + off + e0;
+        float* dk = static_cast<float*>(p.dk) + off + e0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32 / kNH; ++c) {
           float a[32], g[32];
-          tmem_ld32(T_DV + lb + c * 32, a);
-          tmem_ld32(T_DK + lb + c * 32, g);
+          tmem_ld32(T_DV + lq + e0 + c * 32, a);
+          tmem_ld32(T_DK + lq + e0 + c * 32, g);
           tc_wait_ld();
           if (!valid || n_work == 0) continue;
 #pragma unroll
@@ -383,13 +417,13 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
           }
         }
       } else {
-        __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
-        __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
+        __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off + e0;
+        __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off + e0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32 / kNH; ++c) {
           float a[32], g[32];
-          tmem_ld32(T_DV + lb + c * 32, a);
-          tmem_ld32(T_DK + lb + c * 32, g);
+          tmem_ld32(T_DV + lq + e0 + c * 32, a);
+          tmem_ld32(T_DK + lq + e0 + c * 32, g);
           tc_wait_ld();
           if (!valid) continue;
           // A key no query sees gets a zero gradient (TMEM was never written).
@@ -442,8 +476,9 @@ struct DqLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(EwSplit<kEwDq>::kThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   using L = DqLayout<D>;
+  constexpr int kEw = kEwDq, kNH = EwSplit<kEw>::kNH, kCW = EwSplit<kEw>::kCW;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -489,7 +524,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
       mbar_init(BAR_VE(i), 1);
     }
     for (int s = 0; s < 2; ++s) mbar_init(BAR_S(s), 1);
-    mbar_init(BAR_DS, 4);
+    mbar_init(BAR_DS, kEw);
     mbar_init(BAR_DONE, 1);
     mbar_init(BAR_DRAIN, 1);
     mbar_init(BAR_DP, 1);
@@ -568,7 +603,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
         }
         if (!(ok = mbar_wait(BAR_DS, j & 1, abort_flag))) break;
         tc_fence_after();
-        mma_tmem_x_tile<D>(T_DQ, T_S(s), slot_k(j), j > 0);    // dQ += dS K
+        mma_tmem_x_tile<D, kEw>(T_DQ, T_S(s), slot_k(j), j > 0);    // dQ += dS K
         tc_commit(BAR_KE(j % KS));
         if (more) {
           if (!(ok = mbar_wait(BAR_VF((j + 1) % VS), ((j + 1) / VS) & 1, abort_flag))) break;
@@ -583,8 +618,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     }
   } else if (warp >= 4) {
     const int quad = warp & 3;
+    const int grp = (warp - 4) >> 2;  // key columns [grp kCW, (grp+1) kCW)
+    const int g0 = grp * kCW;
     const int r = quad * 32 + lane;  // query row of the tile
-    const uint32_t lb = (uint32_t)(quad * 32) << 16;
+    const uint32_t lq = (uint32_t)(quad * 32) << 16;
+    const uint32_t lb = lq + (uint32_t)g0;
     const long long t = (long long)t0 + r;
     const bool valid = t < p.N_q;
     const long long srow = ((long long)b * p.Hq + h) * p.Npad + t;
@@ -598,25 +636,23 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
       const int s = j & 1;
       if (!(ok = mbar_wait(BAR_S(s), (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      const long long kl = min(klast_abs, p.N_kv - 1) - (long long)j * kBT;
-      const int klast = (int)(kl < -1 ? -1 : (kl > kBT ? kBT : kl));
+      // Last visible column of this group (relative to g0): -1 = none.
+      const long long kl = min(klast_abs, p.N_kv - 1) - (long long)j * kBT - g0;
+      const int klast = (int)(kl < -1 ? -1 : (kl > kCW ? kCW : kl));
       // P first (while dP may still be in the tensor pipe), then dS over S.
-      float pv[kBT];
+      float pv[kCW];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(T_S(s) + lb + c * 32, sv);
-        tc_wait_ld();
+      for (int c = 0; c < kCW / 32; ++c) tmem_ld32(T_S(s) + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
+      tc_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float pe = ex2(fmaf(sv[i], sl, -lse2));
-          pv[c * 32 + i] = c * 32 + i > klast ? 0.f : pe;
-        }
+      for (int i = 0; i < kCW; ++i) {
+        const float pe = ex2(fmaf(pv[i], sl, -lse2));
+        pv[i] = i > klast ? 0.f : pe;
       }
       if (!(ok = mbar_wait(BAR_DP, j & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kCW / 32; ++c) {
         float dp[32];
         tmem_ld32(T_DP + lb + c * 32, dp);
         tc_wait_ld();
@@ -637,14 +673,15 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     if (ok) {
       tc_fence_after();
       const long long off = (((long long)b * p.N_q + (valid ? t : 0)) * p.Hq + h) * D;
+      const int e0 = grp * (D / kNH);  // this warp's dQ columns
       if (p.accumulate) {
         // dq += scale dS K into the caller's float32 row (unchanged when no
         // key of this call is visible to the tile).
-        float* dq = static_cast<float*>(p.dq) + off;
+        float* dq = static_cast<float*>(p.dq) + off + e0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32 / kNH; ++c) {
           float a[32];
-          tmem_ld32(T_DQ + lb + c * 32, a);
+          tmem_ld32(T_DQ + lq + e0 + c * 32, a);
           tc_wait_ld();
           if (!valid || n_jt == 0) continue;
 #pragma unroll
@@ -658,11 +695,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
           }
         }
       } else {
-        __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + off;
+        __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + off + e0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32 / kNH; ++c) {
           float a[32];
-          tmem_ld32(T_DQ + lb + c * 32, a);
+          tmem_ld32(T_DQ + lq + e0 + c * 32, a);
           tc_wait_ld();
           if (!valid) continue;
           // A query that sees no key gets a zero gradient (TMEM never written).
@@ -755,9 +792,9 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if ((e = set_smem_attr<2 * D + 0>(bwd_dkdv_kernel<D>, DkdvLayout<D>::kAlloc)) != cudaSuccess) return e;
   if ((e = set_smem_attr<2 * D + 1>(bwd_dq_kernel<D>, DqLayout<D>::kAlloc)) != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<(unsigned)((long long)prm.n_kt * a.Hkv * a.B), 256, DkdvLayout<D>::kAlloc, st>>>(prm);
+  bwd_dkdv_kernel<D><<<(unsigned)((long long)prm.n_kt * a.Hkv * a.B), EwSplit<kEwDkdv>::kThreads, DkdvLayout<D>::kAlloc, st>>>(prm);
   if ((e = count_launch(cudaGetLastError())) != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<(unsigned)((long long)prm.n_qt * a.Hq * a.B), 256, DqLayout<D>::kAlloc, st>>>(prm);
+  bwd_dq_kernel<D><<<(unsigned)((long long)prm.n_qt * a.Hq * a.B), EwSplit<kEwDq>::kThreads, DqLayout<D>::kAlloc, st>>>(prm);
   return count_launch(cudaGetLastError());
 }
 
