@@ -53,8 +53,8 @@ NCU_TRAFFIC = {
     "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541501e9, "src": "7ee2ab864cd3d8e7"},
     "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541501e9, "src": "7ee2ab864cd3d8e7"},
     # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step (prep + dK/dV + dQ):
-    # 0.541 + 0.011, 1.087 + 0.509, 1.084 + 0.255 GB read + written.
-    "llama7b_prefill_N32768 bwd": {"bytes": 3.487206e9, "src": "e66ff11ce68aa9f4"},
+    # 0.541 + 0.010, 1.084 + 0.508, 1.085 + 0.256 GB read + written.
+    "llama7b_prefill_N32768 bwd": {"bytes": 3.485068e9, "src": "6dd983a4b4a81d8e"},
 }
 
 
