@@ -31,6 +31,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -341,22 +342,32 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
 #pragma unroll
       for (int c = 0; c < kCW / 32; ++c) tmem_ld32(T_ST + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
       tc_wait_ld();
+      // Only warps on the causal diagonal mask columns; the others skip the
+      // selects (a warp-uniform choice, so no lanes diverge).
+      auto p_chunks = [&](auto masked) {
 #pragma unroll
-      for (int c = 0; c < kCW / 32; ++c) {
-        uint32_t up[16];
+        for (int c = 0; c < kCW / 32; ++c) {
+          uint32_t up[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int l0 = c * 32 + i, q0 = g0 + l0;
-          float p0 = ex2(fmaf(pv[l0], sl, -lse2[q0]));
-          float p1 = ex2(fmaf(pv[l0 + 1], sl, -lse2[q0 + 1]));
-          if (q0 < cmin) p0 = 0.f;
-          if (q0 + 1 < cmin) p1 = 0.f;
-          pv[l0] = p0;
-          pv[l0 + 1] = p1;
-          up[i / 2] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 32; i += 2) {
+            const int l0 = c * 32 + i, q0 = g0 + l0;
+            float p0 = ex2(fmaf(pv[l0], sl, -lse2[q0]));
+            float p1 = ex2(fmaf(pv[l0 + 1], sl, -lse2[q0 + 1]));
+            if constexpr (decltype(masked)::value) {
+              if (q0 < cmin) p0 = 0.f;
+              if (q0 + 1 < cmin) p1 = 0.f;
+            }
+            pv[l0] = p0;
+            pv[l0 + 1] = p1;
+            up[i / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(T_ST + lb + c * 16, up);
         }
-        tmem_st16(T_ST + lb + c * 16, up);
-      }
+      };
+      if (__any_sync(0xffffffffu, cmin > g0))
+        p_chunks(std::true_type{});
+      else
+        p_chunks(std::false_type{});
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -644,10 +655,16 @@ __global__ void __launch_bounds__(EwSplit<kEwDq>::kThreads, 1) bwd_dq_kernel(con
 #pragma unroll
       for (int c = 0; c < kCW / 32; ++c) tmem_ld32(T_S(s) + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
       tc_wait_ld();
+      // Warps whose rows see every key of their columns skip the selects.
+      if (__all_sync(0xffffffffu, klast >= kCW - 1)) {
 #pragma unroll
-      for (int i = 0; i < kCW; ++i) {
-        const float pe = ex2(fmaf(pv[i], sl, -lse2));
-        pv[i] = i > klast ? 0.f : pe;
+        for (int i = 0; i < kCW; ++i) pv[i] = ex2(fmaf(pv[i], sl, -lse2));
+      } else {
+#pragma unroll
+        for (int i = 0; i < kCW; ++i) {
+          const float pe = ex2(fmaf(pv[i], sl, -lse2));
+          pv[i] = i > klast ? 0.f : pe;
+        }
       }
       if (!(ok = mbar_wait(BAR_DP, j & 1, abort_flag))) break;
       tc_fence_after();
