@@ -23,10 +23,11 @@
 //                     dQ += dS K in TMEM.
 // Warp roles in both: warp 0 TMA, warp 1 MMA issue (one thread), warp 2
 // TMEM allocation, warps 4.. the elementwise warps.  An elementwise thread
-// owns one TMEM lane (tile row) and one column group: two warps share each
-// lane quarter, one per half of the tile's 128 columns, so two warps per SM
-// sub-partition overlap their exponential chains.  Every mbarrier wait is
-// bounded as in the forward.
+// owns one TMEM lane (tile row) and one column group.  dK/dV runs two warps
+// per lane quarter, one per half of the tile's 128 columns, so two warps per
+// SM sub-partition overlap their exponential chains; dQ runs one warp per
+// quarter over all 128 columns.  Every mbarrier wait is bounded as in the
+// forward.
 #pragma once
 
 #include <cstdlib>
