@@ -499,6 +499,81 @@ def pin_window_anchor(O):
     _close(lc, rlc, 1e-12, "full window = causal (lse)")
 
 
+def _sdpa_rows(q, k, v, causal, scale, cache_idx, rows, heads, chunk=64):
+    """torch float64 SDPA on selected query rows and heads, a few rows per call
+    (rows are independent, so calling the library per group of rows changes
+    nothing but the memory it needs)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    G = Hq // Hkv
+    kpos = torch.arange(k.shape[1])
+    outs, lses = [], []
+    for c0 in range(0, rows.shape[0], chunk):
+        r = torch.from_numpy(rows[c0:c0 + chunk])
+        qs = q[:, r][:, :, heads]
+        hk = [h // G for h in heads]
+        ks, vs = k[:, :, hk], v[:, :, hk]
+        qpos = r + (0 if cache_idx < 0 else cache_idx)
+        mask = (kpos[None, :] <= qpos[:, None]) if causal else torch.ones(r.shape[0], k.shape[1], dtype=torch.bool)
+        o = F.scaled_dot_product_attention(qs.transpose(1, 2), ks.transpose(1, 2), vs.transpose(1, 2),
+                                           attn_mask=mask, scale=scale).transpose(1, 2)
+        sc = (torch.einsum("bqhd,bkhd->bhqk", qs, ks) * scale).masked_fill(~mask, float("-inf"))
+        outs.append(o.numpy())
+        lses.append(torch.logsumexp(sc, dim=-1).numpy())
+    return np.concatenate(outs, axis=1), np.concatenate(lses, axis=2)
+
+
+def pin_row_blocks(O):
+    # attention_ref walks the query rows in blocks of 256 (fewer when a key
+    # row is long).  Cases with several blocks, so that blocks after the
+    # first (r0 > 0) and a ragged last block are written, against float64
+    # SDPA; and the rows= / heads= sample against SDPA's full result sliced.
+    cases = [(1, 600, 600, 4, 2, 4, True, 0.4, -1), (2, 600, 600, 1, 1, 4, False, 0.3, -1),
+             (1, 300, 633, 2, 2, 4, True, 0.5, 333)]
+    for i, (B, N_q, N_kv, Hq, Hkv, d, causal, scale, ci) in enumerate(cases):
+        q = _rand((B, N_q, Hq, d), 240 + i)
+        k = _rand((B, N_kv, Hkv, d), 250 + i)
+        v = _rand((B, N_kv, Hkv, d), 260 + i)
+        ref_o, ref_l = _sdpa_case(q, k, v, causal, scale, ci)
+        o, l = O.attention_ref(q, k, v, causal=causal, scale=scale, cache_idx=ci)
+        _close(o, ref_o, 1e-10, f"row blocks out case {i}")
+        _close(l, ref_l, 1e-10, f"row blocks lse case {i}")
+        rows = np.random.default_rng(i).permutation(N_q)[:290]   # unsorted, two blocks
+        heads = list(range(Hq))[::-1]
+        so, sl = O.attention_ref(q, k, v, causal=causal, scale=scale, cache_idx=ci, rows=rows, heads=heads)
+        _close(so, ref_o[:, rows][:, :, heads], 1e-10, f"sampled rows out case {i}")
+        _close(sl, ref_l[:, heads][:, :, rows], 1e-10, f"sampled rows lse case {i}")
+
+
+def pin_long_key_rows(O):
+    # Key rows longer than 131072 shrink the row block below 256 rows (255
+    # at 131200 keys).  A causal prefill of 131200 tokens on an unsorted
+    # sample of rows spanning two blocks (the second ragged), in reversed
+    # head order, against float64 SDPA per group of rows; then identical
+    # keys, whose result is closed-form: the prefix mean of V and
+    # lse = s + ln(position + 1).
+    B, N, Hq, Hkv, d, scale = 1, 131200, 2, 1, 4, 0.5
+    q = _rand((B, N, Hq, d), 270)
+    k = _rand((B, N, Hkv, d), 271)
+    v = _rand((B, N, Hkv, d), 272)
+    rng = np.random.default_rng(11)
+    rows = np.concatenate([rng.integers(0, N, 296), [0, N - 1, 131071, 131072]])
+    heads = [1, 0]
+    o, l = O.attention_ref(q, k, v, causal=True, scale=scale, rows=rows, heads=heads)
+    ro, rl = _sdpa_rows(q, k, v, True, scale, -1, rows, heads)
+    _close(o, ro, 1e-10, "long key rows out")
+    _close(l, rl, 1e-10, "long key rows lse")
+    k1 = _rand((1, 1, 1, d), 273)
+    kk = k1.expand(B, N, Hkv, d).contiguous()
+    o, l = O.attention_ref(q, kk, v, causal=True, scale=scale, rows=rows, heads=heads[:1])
+    prefix_mean = (np.cumsum(v[0, :, 0].numpy(), axis=0) / np.arange(1, N + 1)[:, None])[rows]
+    for hi, h in enumerate(heads[:1]):
+        s = scale * (q[0, rows, h] @ k1[0, 0, 0]).numpy()
+        _close(o[0, :, hi], prefix_mean, 1e-12, f"long identical keys out head {h}")
+        _close(l[0, hi], s + np.log(rows + 1.0), 1e-12, f"long identical keys lse head {h}")
+
+
 ALL_PINS = [pin_sdpa, pin_bruteforce, pin_closed_forms, pin_ring_equals_full, pin_invariants,
             pin_block_step, pin_lse_merge, pin_schedule, pin_backward_autograd, pin_backward_finite_difference,
-            pin_backward_ring, pin_fp8_decode, pin_fp8kv_attention, pin_window_anchor]
+            pin_backward_ring, pin_fp8_decode, pin_fp8kv_attention, pin_window_anchor, pin_row_blocks,
+            pin_long_key_rows]

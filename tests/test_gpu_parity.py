@@ -269,11 +269,3 @@ def test_exp2_poly_error_bound():
     z = R.ring_attn_exp2_poly(torch.tensor([-200.0, -1e30], device="cuda"))
     assert torch.allclose(z.double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64, device="cuda"),
                           rtol=1e-4, atol=0)
-
-
-@pytest.mark.parametrize("mask", ["0x11", "0x55", "0xff"])
-def test_prefill_with_fma_exp2(monkeypatch, mask):
-    monkeypatch.setenv("RINGATTN_EMU_MASK", mask)
-    check_workload(W(B=1, Hq=4, Hkv=2, N_q=1024, d=128, causal=True, P=4, seed=61))
-    check_workload(W(B=1, Hq=2, Hkv=2, N_q=512, d=64, causal=False, P=2, k_scale=4.0, seed=62))
-    check_workload(W(B=2, Hq=8, Hkv=2, N_q=96, N_kv=2048, cache_idx=1952, d=128, causal=True, P=8, seed=63))
