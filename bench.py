@@ -11,9 +11,15 @@ torch.distributed.run) every rank runs its own seeded copy of the workload
 the timed region is bracketed by barriers and its duration is the maximum
 over ranks.  Rank 0 prints one JSON line.
 
+The default run (config 2, forward) also times the decode-shaped incremental
+queries 5d1 and 5d1f8 (one new token against a 262144-token bf16 or FP8 KV
+cache, at least 100 steps each) and attaches them as the line's "decode"
+list in GB/s against the measured HBM copy bandwidth.
+
 --impl reference times the CPU float64 oracle on this host's cores on a
 bounded sample of the same workload (the reference arm; there is no
-reference GPU implementation).
+reference GPU implementation).  Its ms_per_step is the whole step
+extrapolated from the sampled rate ("extrapolated": true).
 """
 from __future__ import annotations
 
@@ -443,6 +449,36 @@ def oracle_bwd_sample(w, host_qkv, budget_s: float, seed: int = 0):
     return flops, elapsed, done, os.cpu_count()
 
 
+def decode_line(args, key, rank, world, device, peaks, peak_src):
+    """Time one decode-shaped incremental query (the HBM-bound half of the
+    metric) on the same GPU, after the main workload: K+V streamed once per
+    step, reported as algorithmic GB/s against the measured copy bandwidth."""
+    w = workloads.CONFIGS[key]
+    sub = argparse.Namespace(**vars(args))
+    sub.steps = max(100, args.steps)
+    sub.pass_ = "fwd"
+    res = run_ours(sub, w, rank, world, device)
+    ms = res["ms_total"] / sub.steps
+    launch_ms = statistics.mean(res["per_launch_ms"])
+    nbytes = hbm_bytes_of(w)
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    src_hash = kernel_source_hash("decode" if kernel_name(w, False).startswith("decode") else "fwd")
+    tr = NCU_TRAFFIC.get(w.name)
+    return {"workload": w.name, "kv_cache": "fp8 e4m3 + per-head scales" if w.kv_dtype == "fp8" else w.dtype,
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N_q": w.N_q, "N_kv": w.N_kv, "d": w.d,
+            "cache_idx": w.cache_idx, "steps": sub.steps, "warmup": sub.warmup, "ms_per_step": ms,
+            "value": nbytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "tokens_per_s": w.B * w.N_q * world / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": tr["bytes"] if tr and tr.get("src") == src_hash else None,
+                         "peak_source": f"{peak_src} (hbm)", "kernel": kernel_name(w, False),
+                         "algorithmic_per_launch": nbytes},
+            "e2e": {"value": nbytes * world / (res["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+            "gpu_launches": res["launches"], "clocks": res["clocks"]}
+
+
 def host_inputs(w):
     if w.kv_dtype == "fp8":
         return workloads.make_fp8_kv(w, device="cpu")
@@ -461,6 +497,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", default="5d1,5d1f8",
+                    help="decode workloads timed after the forward prefill of config 2 and reported in the "
+                         "line's 'decode' list (comma-separated keys; 'none' to skip)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -500,7 +539,8 @@ def main():
             val = tot_f / tot_s / 1e12
             line = {"impl": "reference", "metric": "attention bwd TFLOP/s", "value": val, "unit": "TFLOP/s",
                     "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                    "ms_per_step": 1e3 * flops / (val * 1e12), "higher_is_better": True, "scaling": "weak",
+                    "ms_per_step": 1e3 * flops / (val * 1e12), "extrapolated": True,
+                    "higher_is_better": True, "scaling": "weak",
                     "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                     "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                      "sample": f"float64 gradient oracle on one KV-head group of the first "
@@ -520,7 +560,8 @@ def main():
         val = tot_f / tot_s / 1e12
         line = {"impl": "reference", "metric": "attention fwd TFLOP/s", "value": val, "unit": "TFLOP/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1e3 * flops / (val * 1e12), "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": 1e3 * flops / (val * 1e12), "extrapolated": True,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                 "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                  "sample": f"{tot_rows} random (row, head) query rows in runs of 16, "
@@ -534,6 +575,10 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     device = local_rank
     res = run_ours(args, w, rank, world, device)
+    decode = None
+    if not bwd and args.config == "2" and args.decode != "none":
+        decode = [decode_line(args, config_key(key), rank, world, device, peaks, peak_src)
+                  for key in args.decode.split(",")]
     ms_step = res["ms_total"] / args.steps
     value = aggregate_tflops(flops, world, ms_step)
     launch_ms = statistics.mean(res["per_launch_ms"])
@@ -587,6 +632,8 @@ def main():
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
     }
+    if decode is not None:
+        line["decode"] = decode
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

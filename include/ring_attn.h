@@ -251,10 +251,17 @@ int ring_attn_bwd_block_step(const void* q_chunk, const void* k_chunk, const voi
  *     ring_attn_last_error(); cache_idx == -1 is rejected the same way;
  *   - the first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture;
+ *   - the looked-up address is kept for the life of the process, so a
+ *     device reset (cudaDeviceReset) after the first call on that device is
+ *     not supported;
  *   - all calls share the one array and it keeps the last call's contents:
  *     calls that may overlap on the GPU (different streams, or different
  *     host threads on the same device) race and must be serialised by the
- *     caller.
+ *     caller;
+ *   - when ring_attn_sync_status() reports RA_ERR_DEVICE_TIMEOUT for the
+ *     stream, out and lse of the calls before it are undefined: a split
+ *     that gave up writes no partial, and the merge may then read the
+ *     previous call's partials from the shared array.
  */
 int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
                           int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
@@ -269,9 +276,10 @@ int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out
 int ring_attn_sync_status(void* stream);
 
 /*
- * ring_attn_exp2_poly -- y[i] = 2^x[i] evaluated the way the bf16 forward
- * evaluates part of its softmax exponentials on FMA units instead of the
- * special-function unit: x = n + f (n = round(x)), 2^f by a degree-3
+ * ring_attn_exp2_poly -- y[i] = 2^x[i] on FMA units instead of the
+ * special-function unit, the polynomial exp2 the bf16 forward can use for a
+ * compile-time share of its softmax exponentials (none by default, since
+ * every share measured was slower): x = n + f (n = round(x)), 2^f by a degree-3
  * minimax polynomial on [-1/2, 1/2] (max relative error 7.5e-5), 2^n by an
  * exponent-field add; inputs below -125 are clamped to -125.  Valid for
  * x <= 127.  Exposed so the polynomial can be checked against the

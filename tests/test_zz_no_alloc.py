@@ -2,16 +2,21 @@
 cannot let the library allocate device memory (their own pool owns the
 budget, or an allocation on a latency-critical path is not acceptable).
 
-It must give the same result as ring_attn_fwd, within the parity tolerance,
-on consecutive calls that share its fixed scratch array; the second call uses
-other inputs and another shape, so stale scratch contents from the first
-call would show up.  This file is collected last on purpose.
+It must give the same result as ring_attn_fwd, and as the float64 oracle,
+within the parity tolerance, on consecutive calls that share its fixed
+scratch array; the second call uses other inputs and another shape, so stale
+scratch contents from the first call would show up.  It must also succeed
+while the allocating path is made to fail (RINGATTN_FAULT=alloc), which shows
+that it never reaches the library's workspace allocation.  This file is
+collected last on purpose.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 from parity_util import TOL_LSE, TOL_OUT
 
@@ -46,6 +51,12 @@ def _check_same(got_out, got_lse, ref_out, ref_lse):
     assert (got_lse - ref_lse).abs().max().item() <= TOL_LSE
 
 
+def _check_oracle(w, q, k, v, got_out, got_lse):
+    ro, rl = oracle.attention_ref(q, k, v, causal=w.causal, scale=w.scale, cache_idx=w.cache_idx)
+    assert np.max(np.abs(got_out.float().cpu().numpy() - ro)) <= TOL_OUT["bf16"]
+    assert np.max(np.abs(got_lse.cpu().numpy() - rl)) <= TOL_LSE
+
+
 def test_noalloc_matches_fwd_on_two_calls_in_a_row():
     R = _ra()
     w1 = workloads.small(B=2, Hq=8, Hkv=2, N_q=4, N_kv=4096, cache_idx=4092, d=128, causal=True, P=16, seed=41)
@@ -58,9 +69,29 @@ def test_noalloc_matches_fwd_on_two_calls_in_a_row():
         assert st == R.RA_OK, R.lib.ring_attn_last_error().decode()
         torch.cuda.synchronize()
         assert R.ring_attn_sync_status() == 0
-        results.append((out, lse, ref_out, ref_lse))
-    for out, lse, ref_out, ref_lse in results:
+        results.append((w, q, k, v, out, lse, ref_out, ref_lse))
+    for w, q, k, v, out, lse, ref_out, ref_lse in results:
         _check_same(out, lse, ref_out, ref_lse)
+        _check_oracle(w, q, k, v, out, lse)
+
+
+def test_noalloc_never_takes_the_allocating_path(monkeypatch):
+    # With RINGATTN_FAULT=alloc every workspace allocation of the library
+    # fails.  A split-KV call of ring_attn_fwd therefore fails with
+    # RA_ERR_OOM, while the allocation-free call, on the same inputs and
+    # split count, succeeds and matches the oracle.
+    R = _ra()
+    w = workloads.small(B=1, Hq=8, Hkv=2, N_q=3, N_kv=4096, cache_idx=4093, d=128, causal=True, P=8, seed=45)
+    q, k, v = _case(w)
+    monkeypatch.setenv("RINGATTN_SPLITS", "4")
+    monkeypatch.setenv("RINGATTN_FAULT", "alloc")
+    with pytest.raises(RuntimeError):
+        R.ring_attn_fwd(q, k, v, causal=w.causal, P=w.P, cache_idx=w.cache_idx, scale=w.scale)
+    st, out, lse = _call_noalloc_c_abi(R, w, q, k, v)
+    assert st == R.RA_OK, R.lib.ring_attn_last_error().decode()
+    torch.cuda.synchronize()
+    assert R.ring_attn_sync_status() == 0
+    _check_oracle(w, q, k, v, out, lse)
 
 
 def test_noalloc_rejects_oversize_and_prefill():
