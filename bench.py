@@ -16,6 +16,11 @@ queries 5d1 and 5d1f8 (one new token against a 262144-token bf16 or FP8 KV
 cache, at least 100 steps each) and attaches them as the line's "decode"
 list in GB/s against the measured HBM copy bandwidth.
 
+--ring times the sequence-parallel ring itself (ring.ring_attention with
+zigzag chunks across the N ranks, KV exchanged between neighbours every
+step; strong scaling at the workload's full sequence) and adds the bytes
+exchanged per step to the line.
+
 --impl reference times the CPU float64 oracle on this host's cores on a
 bounded sample of the same workload (the reference arm; there is no
 reference GPU implementation).  Its ms_per_step is the whole step
@@ -68,9 +73,9 @@ NCU_TRAFFIC = {
 # The kernel families: "fwd" (the general forward), "decode" (the keys-on-M
 # decode kernel, which shares the FP8 converter and cursor code of the
 # forward's sources) and "bwd".
-_NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh", "decode_sm100.cuh"},
+_NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh", "decode_sm100.cuh", "decode_f8_sm100.cuh"},
                 "decode": {"bwd_sm100.cuh", "fwd_simt.cuh"},
-                "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh"}}
+                "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh", "decode_f8_sm100.cuh"}}
 
 
 def kernel_source_hash(pass_: str = "fwd") -> str:
@@ -120,10 +125,13 @@ def kernel_name(w: workloads.Workload, bwd: bool) -> str:
         return "bwd_prep + bwd_dkdv + bwd_dq (whole step)"
     if w.dtype != "bf16":
         return "simt_attn_kernel"
-    fp8 = " (FP8 KV, converter warpgroup)" if w.kv_dtype == "fp8" else ""
-    if w.d == 128 and w.cache_idx > 0 and w.window < 0 and (w.Hq // w.Hkv) * w.N_q <= 16:
-        return "decode_sm100_kernel" + fp8
-    return "fwd_sm100_kernel" + fp8
+    rows = (w.Hq // w.Hkv) * w.N_q
+    if w.d == 128 and w.cache_idx > 0 and w.window < 0:
+        if w.kv_dtype == "fp8" and rows <= 16:
+            return "decode_f8_sm100_kernel (FP8 KV on the 8-bit MMA path)"
+        if w.kv_dtype != "fp8" and rows <= 16:
+            return "decode_sm100_kernel"
+    return "fwd_sm100_kernel" + (" (FP8 KV, converter warpgroup)" if w.kv_dtype == "fp8" else "")
 
 
 def window_anchor_pairs(n: int, window: int, period: int) -> float:
@@ -362,6 +370,82 @@ def run_ours(args, w, rank, world, device):
     return res
 
 
+# ------------------------------------------------------------ the ring itself
+def run_ring(args, w, rank, world, device):
+    """Time ring.ring_attention (sequence-parallel forward) over the ranks.
+
+    The workload's whole sequence is cut into 2 * world chunks; rank i holds
+    chunks i and 2 world - 1 - i (zigzag layout, equal causal work per rank)
+    and exchanges KV with its ring neighbours every step.  Total work is
+    fixed as world grows (strong scaling).  Returns the timing record.
+    """
+    from long_context_exact_blockwise_b200 import ring
+    import long_context_exact_blockwise_b200.ringattn as R
+
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    q, k, v = workloads.make_qkv(w, device=device)  # the same seeded sequence on every rank
+    qc, kc, vc = (ring.shard(x, rank, world, "zigzag") for x in (q, k, v))
+    del q, k, v
+
+    def step():
+        return ring.ring_attention(qc, kc, vc, causal=w.causal, scale=w.scale, layout="zigzag")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if R.ring_attn_sync_status(stream) != 0:
+        raise RuntimeError("device status word set during warm-up")
+    clocks = ClockSampler(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    launches0 = R.ring_attn_launch_count()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        out, lse = step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = R.ring_attn_launch_count() - launches0
+    ms_total = max_over_ranks(t0.elapsed_time(t1), device)
+    # End to end: this rank's chunks from pinned host memory, out and lse back.
+    hq, hk, hv = (x.cpu().pin_memory() for x in (qc, kc, vc))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((qc, hq), (kc, hk), (vc, hv)):
+            dst.copy_(src, non_blocking=True)
+        o, ls = step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(ls, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, args.e2e_steps))
+    a.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, device)
+    kv_bytes_rank = 2 * kc.numel() * kc.element_size()
+    return dict(ms_total=ms_total, launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms,
+                h2d=sum(x.numel() * x.element_size() for x in (hq, hk, hv)),
+                d2h=ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+                exchange_bytes=world * (world - 1) * kv_bytes_rank)
+
+
 # ------------------------------------------------------------ CPU oracle legs
 def oracle_sample(w, host_qkv, budget_s: float, seed: int = 0):
     """Time the float64 oracle on random (row, head) samples of workload w
@@ -497,6 +581,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ring", action="store_true",
+                    help="time ring.ring_attention across the N ranks (sequence-parallel ring, zigzag chunks, "
+                         "strong scaling) instead of data-parallel replicas of the single-GPU kernel")
     ap.add_argument("--decode", default="5d1,5d1f8",
                     help="decode workloads timed after the forward prefill of config 2 and reported in the "
                          "line's 'decode' list (comma-separated keys; 'none' to skip)")
@@ -570,10 +657,36 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
-    if world > 1:
+    if world > 1 or args.ring:
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29533")
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local_rank))
+                                             device_id=torch.device("cuda", local_rank), rank=rank,
+                                             world_size=world)
     device = local_rank
+    if args.ring:
+        if bwd or w.cache_idx >= 0 or w.dtype != "bf16" or w.kv_dtype != "bf16" or w.window >= 0:
+            raise SystemExit("--ring times the bf16 prefill forward")
+        res = run_ring(args, w, rank, world, device)
+        ms_step = res["ms_total"] / args.steps
+        value = flops / (ms_step * 1e-3) / 1e12
+        config["parallelism"] = f"sequence-parallel ring x{world} (zigzag chunks)"
+        config["global_batch"] = w.B
+        line = {"metric": "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": config,
+                "tokens_per_s": w.B * w.N_q / (ms_step * 1e-3),
+                "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
+                "exchange_bytes_per_step": res["exchange_bytes"],
+                "e2e": {"value": flops / (res["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": res["h2d"] * world, "d2h_bytes_per_step": res["d2h"] * world},
+                "gpu_launches": res["launches"], "clocks": res["clocks"]}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+        return
     res = run_ours(args, w, rank, world, device)
     decode = None
     if not bwd and args.config == "2" and args.decode != "none":

@@ -178,8 +178,11 @@ int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, 
  * and out / lse are exact attention over them, as ring_attn_fwd computes
  * them (q, out bf16; lse float32; same shapes, causal, chunk, P, cache_idx
  * and scale rules; incremental queries use split-KV partials and a stream-
- * ordered workspace).  The tensor cores read the codes decoded to bf16,
- * which is exact for every E4M3 value.  Scales must be finite with
+ * ordered workspace).  Decode-shaped blocks (d = 128, at most 16 packed
+ * query rows per KV head) use the tensor cores' 8-bit path with the codes as
+ * operands (the bf16 queries and the probabilities each split exactly into
+ * two E4M3 planes); other shapes read the codes decoded to bf16, which is
+ * exact for every E4M3 value.  Scales must be finite with
  * |k_scale| * scale < 177 (any usable logit range).  All pointers are device memory
  * owned by the caller; q, k8, v8, out 16-byte aligned.  Returns RA_OK,
  * RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA or RA_ERR_OOM.
@@ -267,6 +270,22 @@ int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out
                           int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
                           int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
                           void* stream);
+
+/*
+ * ring_attn_add_and_clear -- acc[i] += part[i], then part[i] = 0, for n
+ * float32 elements: folds one ring visit's dk / dv share, computed by
+ * ring_attn_bwd_block_step into a zeroed buffer `part`, into the
+ * accumulators that travel the ring with their KV chunk (the Ring Attention
+ * page's blockwise loop, §3.1, whose KV moves while the current block is
+ * computed, §3.2).  Computing the share into `part` lets a visit run while
+ * the accumulators it will add into are still in flight; the clear leaves
+ * `part` ready for the next visit.  acc and part: distinct device buffers
+ * owned by the caller, 4-byte aligned (16-byte alignment of both takes the
+ * vector path).  n = 0 is a no-op.  Returns RA_OK, RA_ERR_INVALID_ARG
+ * (null or equal pointers, n < 0, misalignment), RA_ERR_UNSUPPORTED or
+ * RA_ERR_CUDA.
+ */
+int ring_attn_add_and_clear(float* acc, float* part, int64_t n, void* stream);
 
 /*
  * ring_attn_sync_status -- synchronise `stream`, then read and clear the

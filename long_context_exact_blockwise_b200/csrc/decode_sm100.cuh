@@ -624,12 +624,21 @@ CUresult encode_map_box(CUtensorMap* m, const void* base, int d, int H, long lon
 
 }  // namespace
 
+// The FP8-cache decode on the 8-bit MMA path (decode_f8_sm100.cuh).
+cudaError_t launch_decode_f8_sm100(const DecParams& prm, int NR, int mode, long long grid, cudaStream_t st);
+
+// FP8 caches go to the 8-bit MMA kernel (1) or to the converter variant of
+// this kernel (0).
+#ifndef RA_DEC8_NATIVE
+#define RA_DEC8_NATIVE 1
+#endif
+
 // Rows per KV head of an incremental-query block (G heads x N_q tokens) that
-// the keys-on-M decode kernel takes: 16 or 32 (0: it does not apply).
+// the keys-on-M decode kernels take: 16 or 32 (0: they do not apply).
 int decode_rows(const ProblemArgs& a, int mode) {
   if (mode == kModeState || a.d != kDecD || a.wa_period > 0 || a.q_pos0 <= 0) return 0;
   // RINGATTN_DECODE: "0" never; "all" up to 32 rows; default up to 16 rows
-  // (at 32 rows the general kernel measured faster).
+  // (at 32 rows the general kernel measured faster, for both cache types).
   const char* ov = std::getenv("RINGATTN_DECODE");
   if (ov && ov[0] == '0') return 0;
   const bool all = ov && std::strcmp(ov, "all") == 0;
@@ -684,6 +693,7 @@ cudaError_t launch_decode_sm100(const ProblemArgs& a, int mode, cudaStream_t st)
     prm.skip_loads = (f && std::strcmp(f, "device_wait") == 0) ? 1 : 0;
   }
   const long long grid = (long long)a.B * a.Hkv * prm.n_qblk * prm.S;
+  if (a.kv8 && RA_DEC8_NATIVE) return launch_decode_f8_sm100(prm, NR, mode, grid, st);
   if (a.kv8) {
     if (NR == 16)
       return mode == kModeSplit ? launch_dec_cfg<16, RA_DEC8_NSLOT, kModeSplit, RA_DEC8_NSLOT8>(prm, grid, st)

@@ -110,6 +110,9 @@ struct BwdArgs {
 };
 cudaError_t launch_bwd_sm100(const BwdArgs& a, cudaStream_t stream);
 
+// dst += src, then src = 0 (float32, n elements).
+cudaError_t launch_add_clear(float* dst, float* src, long long n, int num_sms, cudaStream_t stream);
+
 // y = exp2_poly2(x) elementwise (the FMA-pipe exp2 of the softmax), for tests.
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 

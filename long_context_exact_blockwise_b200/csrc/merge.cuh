@@ -144,7 +144,43 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
   }
 }
 
+// dst += src, then src = 0, over n floats: 16-byte vectors over the first
+// n4 * 4 elements (n4 = 0 when a pointer is not 16-byte aligned), then the
+// scalar tail.  Grid-stride.
+__global__ void add_clear_kernel(float* __restrict__ dst, float* __restrict__ src, long long n, long long n4) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  float4* d4 = reinterpret_cast<float4*>(dst);
+  float4* s4 = reinterpret_cast<float4*>(src);
+  for (long long i = t0; i < n4; i += stride) {
+    float4 a = d4[i];
+    const float4 b = s4[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    d4[i] = a;
+    s4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (long long i = 4 * n4 + t0; i < n; i += stride) {
+    dst[i] += src[i];
+    src[i] = 0.f;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_add_clear(float* dst, float* src, long long n, int num_sms, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const bool vec = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0;
+  const long long n4 = vec ? n / 4 : 0;
+  const long long work = n4 + (n - 4 * n4);
+  long long blocks = (work + 255) / 256;
+  const long long cap = 4LL * num_sms;  // a few resident blocks per SM, grid-stride beyond
+  if (blocks > cap) blocks = cap;
+  add_clear_kernel<<<(unsigned)blocks, 256, 0, st>>>(dst, src, n, n4);
+  return count_launch(cudaGetLastError());
+}
 
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;

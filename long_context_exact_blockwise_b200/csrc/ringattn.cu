@@ -15,6 +15,7 @@
 // shared without relocatable device code).
 #include "fwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "decode_f8_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "fwd_simt.cuh"
 #include "merge.cuh"
@@ -466,6 +467,18 @@ int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
   if (r != RA_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return finish(launch_exp2_poly(x, y, n, st), st, "ring_attn_exp2_poly");
+}
+
+int ring_attn_add_and_clear(float* acc, float* part, int64_t n, void* stream) {
+  if (n < 0) return RA_ERR_INVALID_ARG;
+  if (n == 0) return RA_OK;
+  if (!acc || !part || acc == part) return RA_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(acc) | reinterpret_cast<uintptr_t>(part)) & 3u) != 0) return RA_ERR_INVALID_ARG;
+  int num_sms = 148;
+  int r = check_device(&num_sms);
+  if (r != RA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return finish(launch_add_clear(acc, part, n, num_sms, st), st, "ring_attn_add_and_clear");
 }
 
 }  // extern "C"

@@ -3,22 +3,36 @@
 The pages' ring ("Ring Attention: the secret of million-token context", §2.1
 chunking, §2.2 ring schedule figure, §3.1 two-level loop, §3.2 overlap of
 the next KV transfer with the current block's compute): the sequence is cut
-into P = world-size chunks; rank i holds Q_i, K_i, V_i and owns output
-rows i.  At step s rank i folds KV chunk (i + s) mod P into its running
-(acc, m, l) state with ``ring_attn_block_step``, while the chunk it will
-need at step s + 1 is received from rank i + 1 and the chunk it holds is
-sent to rank i - 1 (double-buffered point-to-point messages).  After P
-steps ``ring_attn_finalize`` normalises the state once over all keys.
+into chunks spread over the P = world-size ranks; rank i holds its chunks of
+Q, K, V and owns their output rows.  At step s rank i folds the KV chunks of
+rank (i + s) mod P into its running (acc, m, l) state with
+``ring_attn_block_step``, while the KV it will need at step s + 1 is
+received from rank i + 1 and the KV it holds is sent to rank i - 1
+(double-buffered point-to-point messages).  After P steps
+``ring_attn_finalize`` normalises the state once over all keys.  There is no
+output collective.
 
-Causal visits whose keys all lie in the future of the rank's queries change
-nothing and are skipped on the host.  There is no output collective.
+Chunk layouts:
+  - "contiguous": P chunks; rank i holds chunk i.  Under causal masking
+    rank i then does i + 1 non-empty visits, so the last rank does P times
+    the work of the first.
+  - "zigzag": 2P chunks; rank i holds chunks i and 2P - 1 - i (its q, k and
+    v are those two chunks concatenated along the sequence).  Every rank's
+    causal work is then the same (the pages ask for load balancing across
+    the ring: "RingAttention vs RAG", §2.1, dynamic load balancing).
+Causal visits whose keys all lie in the future of a query chunk change
+nothing and are skipped on the host.
 
 The backward (``ring_attention_bwd``) runs the same ring: rank i adds each
 visit's share of dq into its own accumulator with
 ``ring_attn_bwd_block_step``, while the float32 dK / dV accumulators of the
-KV chunk it holds travel with that chunk, one hop per step, after the
-visit's compute.  After P steps every chunk's accumulators have visited
-every rank and the last hop hands them to the chunk's owner.
+KV it holds travel with that KV, one hop per step.  The hop overlaps the
+next visit: that visit's dK / dV share is computed into a zeroed scratch
+buffer while the accumulators are in flight, then folded into them on
+arrival (``ring_attn_add_and_clear``) and sent on.  Every hop is one batch
+of a send and a receive on every rank, so no rank's receive waits behind its
+own send.  After P hops every chunk's accumulators have visited every rank
+and the last hop hands them to the chunk's owner.
 
 The per-visit compute and the final normalisation are injectable so the
 communication protocol can be exercised on CPU ranks (gloo) with any
@@ -28,10 +42,12 @@ library's CUDA kernels.
 from __future__ import annotations
 
 import math
-from typing import Callable, Optional, Tuple
+from typing import Callable, List, Optional, Tuple
 
 import torch
 import torch.distributed as dist
+
+LAYOUTS = ("contiguous", "zigzag")
 
 
 def _default_block_step(q, k, v, q_off, k_off, acc, m, l, *, causal, scale):
@@ -42,6 +58,11 @@ def _default_block_step(q, k, v, q_off, k_off, acc, m, l, *, causal, scale):
 def _default_block_step_bwd(q, k, v, out, dout, lse, q_off, k_off, dq, dk, dv, *, causal, scale):
     from . import ringattn
     ringattn.ring_attn_bwd_block_step(q, k, v, out, dout, lse, q_off, k_off, dq, dk, dv, causal=causal, scale=scale)
+
+
+def _default_add_and_clear(acc, part):
+    from . import ringattn
+    ringattn.ring_attn_add_and_clear(acc, part)
 
 
 def _default_finalize(acc, m, l, out_dtype):
@@ -57,119 +78,179 @@ def _default_init_state(B, Hq, Lq, d, device):
 
 
 def ring_visit_order(rank: int, world: int) -> list:
-    """KV chunk held by `rank` at each step s: (rank + s) mod world."""
+    """Rank whose KV `rank` holds at each step s: (rank + s) mod world."""
     return [(rank + s) % world for s in range(world)]
 
 
+def chunk_ids(rank: int, world: int, layout: str = "contiguous") -> List[int]:
+    """Global chunk indices held by `rank`, in the order they are concatenated:
+    [rank] of `world` chunks ("contiguous"), or [rank, 2 world - 1 - rank] of
+    2 world chunks ("zigzag")."""
+    if layout == "contiguous":
+        return [rank]
+    if layout == "zigzag":
+        return [rank, 2 * world - 1 - rank]
+    raise ValueError(f"layout must be one of {LAYOUTS}")
+
+
+def shard(x: torch.Tensor, rank: int, world: int, layout: str = "contiguous", dim: int = 1) -> torch.Tensor:
+    """This rank's part of a full-sequence tensor (sequence along `dim`) under `layout`."""
+    n = world * (1 if layout == "contiguous" else 2)
+    if x.shape[dim] % n != 0:
+        raise ValueError(f"sequence length {x.shape[dim]} is not a multiple of {n} chunks")
+    L = x.shape[dim] // n
+    return torch.cat([x.narrow(dim, c * L, L) for c in chunk_ids(rank, world, layout)], dim=dim).contiguous()
+
+
+def _pieces(x: torch.Tensor, n: int, dim: int = 1) -> List[torch.Tensor]:
+    L = x.shape[dim] // n
+    return [x.narrow(dim, i * L, L).contiguous() for i in range(n)]
+
+
+def _peers(group, world, rank):
+    send_to = (rank - 1) % world      # the rank that needs our KV next
+    recv_from = (rank + 1) % world    # the rank holding the KV we need next
+    if group is not None:
+        return dist.get_global_rank(group, send_to), dist.get_global_rank(group, recv_from)
+    return send_to, recv_from
+
+
+def _exchange(send: List[torch.Tensor], recv: List[torch.Tensor], g_send: int, g_recv: int, group, tag: int):
+    ops = [dist.P2POp(dist.isend, t, g_send, group, tag + i) for i, t in enumerate(send)]
+    ops += [dist.P2POp(dist.irecv, t, g_recv, group, tag + i) for i, t in enumerate(recv)]
+    return dist.batch_isend_irecv(ops) if ops else []
+
+
 def ring_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
-                   scale: Optional[float] = None, group=None,
+                   scale: Optional[float] = None, group=None, layout: str = "contiguous",
                    block_step: Optional[Callable] = None,
                    finalize: Optional[Callable] = None,
                    init_state: Optional[Callable] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Exact attention for this rank's query chunk over the whole sequence.
+    """Exact attention for this rank's query chunks over the whole sequence.
 
-    q: [B, L, Hq, d] (chunk ``rank`` of the query sequence); k, v:
-    [B, L, Hkv, d] (chunk ``rank`` of the KV sequence).  All ranks hold
-    chunks of the same length L.  Returns (out [B, L, Hq, d], lse
-    [B, Hq, L]) for this rank's rows.  Every rank must call this with the
-    same shapes; the group defaults to the world.
+    q: [B, L, Hq, d]; k, v: [B, L, Hkv, d]: this rank's chunks under
+    `layout` (``shard`` cuts them from full tensors).  Every rank holds the
+    same L.  Returns (out [B, L, Hq, d], lse [B, Hq, L]) for this rank's rows,
+    in the same chunk order.  Every rank must call this with the same shapes
+    and layout; the group defaults to the world.
     """
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     B, L, Hq, d = q.shape
     if k.shape[1] != L or v.shape != k.shape:
         raise ValueError("every rank must hold equal-length q, k, v chunks")
+    n = len(chunk_ids(rank, world, layout))
+    if L % n != 0:
+        raise ValueError(f"the {layout} layout needs a chunk length divisible by {n}")
+    Lp = L // n
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     block_step = block_step or _default_block_step
     finalize = finalize or _default_finalize
     init_state = init_state or _default_init_state
+    g_send, g_recv = _peers(group, world, rank)
 
-    send_to = (rank - 1) % world      # the rank that needs our chunk next
-    recv_from = (rank + 1) % world    # the rank holding the chunk we need next
-    g_send = dist.get_global_rank(group, send_to) if group is not None else send_to
-    g_recv = dist.get_global_rank(group, recv_from) if group is not None else recv_from
-
-    acc, m, l = init_state(B, Hq, L, d, q.device)
-    # The caller's chunks are only read (sent at step 0); received chunks go
-    # to two buffers owned here, used alternately.
-    cur_k, cur_v = k.contiguous(), v.contiguous()
-    bufs = [(torch.empty_like(cur_k), torch.empty_like(cur_v)) for _ in range(min(2, world - 1))]
-    q_off = rank * L
-    for s, j in enumerate(ring_visit_order(rank, world)):
-        reqs = []
-        if s + 1 < world:
-            nxt_k, nxt_v = bufs[s % 2]
-            ops = [dist.P2POp(dist.isend, cur_k, g_send, group),
-                   dist.P2POp(dist.isend, cur_v, g_send, group),
-                   dist.P2POp(dist.irecv, nxt_k, g_recv, group),
-                   dist.P2POp(dist.irecv, nxt_v, g_recv, group)]
-            reqs = dist.batch_isend_irecv(ops)
-        k_off = j * L
-        # A causal visit whose first key is past every query of this chunk
-        # leaves the state unchanged: skip it.
-        if not (causal and k_off > q_off + L - 1):
-            block_step(q, cur_k, cur_v, q_off, k_off, acc, m, l, causal=causal, scale=scale)
+    q_p = _pieces(q, n)
+    q_ids = chunk_ids(rank, world, layout)
+    states = [init_state(B, Hq, Lp, d, q.device) for _ in range(n)]
+    # The held KV as n pieces; received KV goes to two buffer sets owned here.
+    cur = _pieces(k, n) + _pieces(v, n)
+    bufs = [[torch.empty_like(t) for t in cur] for _ in range(min(2, world - 1))]
+    for s, owner in enumerate(ring_visit_order(rank, world)):
+        reqs = _exchange(cur, bufs[s % 2], g_send, g_recv, group, 0) if s + 1 < world else []
+        for ki, kc in enumerate(chunk_ids(owner, world, layout)):
+            k_off = kc * Lp
+            for qi, qc in enumerate(q_ids):
+                q_off = qc * Lp
+                # A causal visit whose first key is past every query of the
+                # chunk leaves its state unchanged: skip it.
+                if causal and k_off > q_off + Lp - 1:
+                    continue
+                block_step(q_p[qi], cur[ki], cur[n + ki], q_off, k_off, *states[qi], causal=causal, scale=scale)
         for r in reqs:
             r.wait()
         if s + 1 < world:
-            cur_k, cur_v = bufs[s % 2]
-    return finalize(acc, m, l, q.dtype)
+            cur = bufs[s % 2]
+    outs = [finalize(*st, q.dtype) for st in states]
+    if n == 1:
+        return outs[0]
+    return torch.cat([o for o, _ in outs], dim=1), torch.cat([ls for _, ls in outs], dim=2)
 
 
 def ring_attention_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
                        lse: torch.Tensor, *, causal: bool, scale: Optional[float] = None, group=None,
-                       block_step_bwd: Optional[Callable] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                       layout: str = "contiguous",
+                       block_step_bwd: Optional[Callable] = None,
+                       add_and_clear: Optional[Callable] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients of ``ring_attention`` for this rank's chunks.
 
-    q, out, dout: [B, L, Hq, d] and lse [B, Hq, L] (this rank's query chunk
-    and the forward's results for it); k, v: [B, L, Hkv, d] (this rank's KV
-    chunk).  Returns (dq, dk, dv) for this rank's chunks, in the input dtypes.
-    Every rank must call this with the same shapes.
+    q, out, dout: [B, L, Hq, d] and lse [B, Hq, L] (this rank's query chunks
+    and the forward's results for them); k, v: [B, L, Hkv, d] (this rank's KV
+    chunks), all under `layout`.  Returns (dq, dk, dv) for this rank's chunks,
+    in the input dtypes.  Every rank must call this with the same shapes.
     """
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     B, L, Hq, d = q.shape
     if k.shape[1] != L or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape:
         raise ValueError("every rank must hold equal-length q, k, v, out, dout chunks")
+    n = len(chunk_ids(rank, world, layout))
+    if L % n != 0:
+        raise ValueError(f"the {layout} layout needs a chunk length divisible by {n}")
+    Lp = L // n
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     block_step_bwd = block_step_bwd or _default_block_step_bwd
+    add_and_clear = add_and_clear or _default_add_and_clear
     acc_dtype = torch.float64 if q.dtype == torch.float64 else torch.float32
+    g_send, g_recv = _peers(group, world, rank)
 
-    send_to = (rank - 1) % world
-    recv_from = (rank + 1) % world
-    g_send = dist.get_global_rank(group, send_to) if group is not None else send_to
-    g_recv = dist.get_global_rank(group, recv_from) if group is not None else recv_from
-
-    dq = torch.zeros(q.shape, device=q.device, dtype=acc_dtype)
-    # Accumulators of the KV chunk held now, and a buffer for the next ones.
-    acc = [torch.zeros(k.shape, device=k.device, dtype=acc_dtype) for _ in range(2)]
-    acc_next = [torch.empty_like(a) for a in acc] if world > 1 else None
-    cur_k, cur_v = k.contiguous(), v.contiguous()
-    bufs = [(torch.empty_like(cur_k), torch.empty_like(cur_v)) for _ in range(min(2, world - 1))]
-    q_off = rank * L
-    for s, j in enumerate(ring_visit_order(rank, world)):
-        reqs = []
-        if s + 1 < world:
-            nxt_k, nxt_v = bufs[s % 2]
-            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_k, g_send, group),
-                                           dist.P2POp(dist.isend, cur_v, g_send, group),
-                                           dist.P2POp(dist.irecv, nxt_k, g_recv, group),
-                                           dist.P2POp(dist.irecv, nxt_v, g_recv, group)])
-        k_off = j * L
-        if not (causal and k_off > q_off + L - 1):
-            block_step_bwd(q, cur_k, cur_v, out, dout, lse, q_off, k_off, dq, acc[0], acc[1], causal=causal,
-                           scale=scale)
+    q_ids = chunk_ids(rank, world, layout)
+    q_p, o_p, do_p = _pieces(q, n), _pieces(out, n), _pieces(dout, n)
+    lse_p = _pieces(lse, n, dim=2)
+    dq_p = [torch.zeros(x.shape, device=x.device, dtype=acc_dtype) for x in q_p]
+    cur = _pieces(k, n) + _pieces(v, n)
+    bufs = [[torch.empty_like(t) for t in cur] for _ in range(min(2, world - 1))]
+    # dK / dV accumulators of the held KV (n pieces each).  With more than
+    # one rank two sets alternate: each hop sends one and receives into the
+    # other, and is waited for (once) before the next hop is posted.  From
+    # step 1 on a visit's share goes to `scratch` (zero) while the
+    # accumulators it adds into are in flight, and is folded into them once
+    # they have arrived.
+    accs = [[torch.zeros(t.shape, device=t.device, dtype=acc_dtype) for t in cur]]
+    if world > 1:
+        accs.append([torch.empty_like(t) for t in accs[0]])
+        scratch = [torch.zeros_like(t) for t in accs[0]]
+    hop = []  # the previous step's accumulator hop (send + receive)
+    a = 0
+    for s, owner in enumerate(ring_visit_order(rank, world)):
+        reqs = _exchange(cur, bufs[s % 2], g_send, g_recv, group, 0) if s + 1 < world else []
+        target = accs[a] if s == 0 else scratch
+        for ki, kc in enumerate(chunk_ids(owner, world, layout)):
+            k_off = kc * Lp
+            for qi, qc in enumerate(q_ids):
+                q_off = qc * Lp
+                if causal and k_off > q_off + Lp - 1:
+                    continue
+                block_step_bwd(q_p[qi], cur[ki], cur[n + ki], o_p[qi], do_p[qi], lse_p[qi], q_off, k_off, dq_p[qi],
+                               target[ki], target[n + ki], causal=causal, scale=scale)
+        if world > 1:
+            if s > 0:
+                for r in hop:
+                    r.wait()
+                for acc_t, part in zip(accs[a], scratch):
+                    add_and_clear(acc_t, part)
+            # The accumulators follow their KV to rank - 1 (the last hop
+            # brings this rank's own chunks home) and the next ones arrive
+            # from rank + 1, in one batch on every rank; the next visit runs
+            # while it is in flight.
+            hop = _exchange(accs[a], accs[1 - a], g_send, g_recv, group, 2 * n)
+            a = 1 - a
         for r in reqs:
             r.wait()
-        if world > 1:
-            # The accumulators follow their chunk to rank - 1; the last hop
-            # brings this rank's own chunk home.
-            for r in dist.batch_isend_irecv([dist.P2POp(dist.isend, acc[0], g_send, group),
-                                             dist.P2POp(dist.isend, acc[1], g_send, group),
-                                             dist.P2POp(dist.irecv, acc_next[0], g_recv, group),
-                                             dist.P2POp(dist.irecv, acc_next[1], g_recv, group)]):
-                r.wait()
-            acc, acc_next = acc_next, acc
         if s + 1 < world:
-            cur_k, cur_v = bufs[s % 2]
-    return dq.to(q.dtype), acc[0].to(k.dtype), acc[1].to(v.dtype)
+            cur = bufs[s % 2]
+    for r in hop:
+        r.wait()
+    dk = torch.cat(accs[a][:n], dim=1) if n > 1 else accs[a][0]
+    dv = torch.cat(accs[a][n:], dim=1) if n > 1 else accs[a][n]
+    dq = torch.cat(dq_p, dim=1) if n > 1 else dq_p[0]
+    return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype)

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "RingAttnError", "lib", "LIB_PATH",
     "ring_attn_fwd", "ring_attn_fwd_f32", "ring_attn_fwd_noalloc", "ring_attn_fwd_fp8kv", "ring_attn_fwd_window_anchor", "ring_attn_bwd", "ring_attn_bwd_block_step", "ring_attn_block_step", "ring_attn_finalize",
-    "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly",
+    "lse_merge", "ring_attn_sync_status", "ring_attn_error_string", "ring_attn_version", "ring_attn_launch_count", "ring_attn_exp2_poly", "ring_attn_add_and_clear",
     "ring_attn", "init_state",
     "RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED", "RA_ERR_CUDA", "RA_ERR_DEVICE_TIMEOUT",
     "RA_ERR_OOM", "RA_DTYPE_BF16", "RA_DTYPE_F32",
@@ -67,6 +67,7 @@ _SIGS = {
     "ring_attn_version": [],
     "ring_attn_launch_count": [],
     "ring_attn_exp2_poly": [_p, _p, _l, _p],
+    "ring_attn_add_and_clear": [_p, _p, _l, _p],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -121,6 +122,18 @@ def ring_attn_exp2_poly(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
     y = torch.empty_like(x) if out is None else out
     _check(lib.ring_attn_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream, x.device)), "ring_attn_exp2_poly")
     return y
+
+
+def ring_attn_add_and_clear(acc: torch.Tensor, part: torch.Tensor, stream=None) -> torch.Tensor:
+    """acc += part, then part = 0 (float32, same shape): folds one ring
+    visit's dk / dv share into the accumulators travelling the ring."""
+    _need(acc, "acc", torch.float32)
+    _need(part, "part", torch.float32)
+    if acc.shape != part.shape or acc.device != part.device:
+        raise ValueError("acc and part must have the same shape and device")
+    _check(lib.ring_attn_add_and_clear(_ptr(acc), _ptr(part), acc.numel(), _stream(stream, acc.device)),
+           "ring_attn_add_and_clear")
+    return acc
 
 
 def ring_attn_launch_count() -> int:

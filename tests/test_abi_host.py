@@ -160,3 +160,14 @@ def test_window_anchor_validation():
     for i, val in ((12, -1), (13, 0), (13, 100), (13, 384), (9, 96), (10, 100)):
         bad = list(ok_args); bad[i] = val
         assert L.ring_attn_fwd_window_anchor(*bad) == ra.RA_ERR_INVALID_ARG, (i, val)
+
+
+def test_add_and_clear_validation():
+    ra = _lib()
+    L = ra.lib
+    assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20000), 64, None) == ra.RA_ERR_UNSUPPORTED  # no GPU
+    assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20000), 0, None) == ra.RA_OK
+    assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20000), -1, None) == ra.RA_ERR_INVALID_ARG
+    assert L.ring_attn_add_and_clear(None, FAKE, 8, None) == ra.RA_ERR_INVALID_ARG
+    assert L.ring_attn_add_and_clear(FAKE, FAKE, 8, None) == ra.RA_ERR_INVALID_ARG  # the same buffer twice
+    assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20002), 8, None) == ra.RA_ERR_INVALID_ARG  # unaligned

@@ -1,9 +1,11 @@
 """Forward over an FP8 (E4M3) KV cache on the GPU against the float64 oracle.
 
 The oracle attends over the dequantised cache (codes decoded by the format's
-definition, times the per-(batch, KV head) scales); the kernel decodes the
-codes to bf16 (exact) in shared memory and folds the scales into the score
-scale and the final normalisation.  Tolerances are the bf16 path's.
+definition, times the per-(batch, KV head) scales).  Decode-shaped blocks
+(d = 128, at most 32 packed rows per KV head) run on the 8-bit MMA path with
+the codes as operands; other shapes decode the codes to bf16 (exact) in
+shared memory.  Both fold the scales into the score scale and the final
+normalisation.  Tolerances are the bf16 path's.
 """
 import numpy as np
 import pytest
@@ -50,11 +52,13 @@ def test_fp8kv_matches_oracle(B, Hq, Hkv, N_q, N_kv, ci, d, causal, P):
 
 
 def test_fp8kv_equals_bf16_path_on_the_decoded_cache():
-    # With power-of-two scales the FP8 kernel and the bf16 kernel on the
-    # decoded cache do the same float operations in the same order: the
-    # results must agree bit for bit (this checks the decode and its layout).
+    # With power-of-two scales the converter kernel (FP8 codes decoded to bf16
+    # in shared memory) and the bf16 kernel on the decoded cache do the same
+    # float operations in the same order: the results must agree bit for bit
+    # (this checks the decode and its layout).  16 tokens x 4 heads = 64
+    # packed rows: more than the 8-bit decode kernel takes.
     R = ra()
-    w = workloads.small(B=2, Hq=8, Hkv=2, N_q=4, N_kv=2048, cache_idx=2044, d=128, causal=True, P=4, seed=650,
+    w = workloads.small(B=2, Hq=8, Hkv=2, N_q=16, N_kv=2048, cache_idx=2032, d=128, causal=True, P=4, seed=650,
                         kv_dtype="fp8")
     q, k8, v8, _, _ = workloads.make_fp8_kv(w, device="cuda")
     sc = torch.full((w.B, w.Hkv), 2.0 ** -6, device="cuda")

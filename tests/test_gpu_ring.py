@@ -56,3 +56,21 @@ def test_ring_driver_cuda_backward(one_rank_group, causal):
     for got, r in zip((dq, dk, dv), ref):
         g = got.float().cpu().numpy()
         assert np.all(np.abs(g - r) <= 2e-2 + 2e-2 * np.abs(r))
+
+
+@pytest.mark.parametrize("n,offset", [(1, 0), (7, 0), (4096 * 3 + 5, 0), (1000, 1), (12345, 3)])
+def test_add_and_clear(n, offset):
+    # acc += part, part = 0, on 16-byte aligned buffers (vector path and a
+    # tail) and on buffers offset by 1 or 3 floats (scalar path).
+    import long_context_exact_blockwise_b200.ringattn as R
+    g = torch.Generator(device="cuda").manual_seed(n)
+    acc_full = torch.randn(n + offset, generator=g, device="cuda")
+    part_full = torch.randn(n + offset, generator=g, device="cuda")
+    acc, part = acc_full[offset:], part_full[offset:]
+    want = (acc.double() + part.double()).float()
+    before_head = acc_full[:offset].clone()
+    R.lib.ring_attn_add_and_clear(acc.data_ptr(), part.data_ptr(), n, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, want)
+    assert torch.count_nonzero(part).item() == 0
+    assert torch.equal(acc_full[:offset], before_head)

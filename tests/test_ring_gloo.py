@@ -45,55 +45,69 @@ def _oracle_compute():
     return block_step, finalize, init_state
 
 
-def _worker(rank, world, port, case, results):
+CASES = [(1, 2, 2, 16, 8, True), (2, 4, 2, 12, 8, False), (1, 4, 1, 10, 4, True)]
+LAYOUTS = ["contiguous", "zigzag"]
+
+
+def _setup(rank, world, port):
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     sys.path.insert(0, root)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
+
+
+def _worker(rank, world, port, results):
+    _setup(rank, world, port)
     try:
         import oracle
         import workloads
-        from long_context_exact_blockwise_b200.ring import ring_attention
+        from long_context_exact_blockwise_b200.ring import ring_attention, shard
 
-        B, Hq, Hkv, L, d, causal = case
-        w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
-                            seed=11 + world)
-        q, k, v = workloads.make_qkv(w)
-        q, k, v = q.double(), k.double(), v.double()
-        sl = slice(rank * L, (rank + 1) * L)
-        bs, fin, init = _oracle_compute()
-        qc, kc, vc = q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous()
-        before = [x.clone() for x in (qc, kc, vc)]
-        out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, block_step=bs, finalize=fin,
-                                  init_state=init)
-        # The ring only reads the caller's chunks.
-        assert all(torch.equal(a, b) for a, b in zip(before, (qc, kc, vc)))
-        ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
-        err_o = float(np.max(np.abs(out.numpy() - ro[:, sl])))
-        err_l = float(np.max(np.abs(lse.numpy() - rl[:, :, sl])))
-        results[rank] = (err_o, err_l)
+        # Every case and layout in one process group (every rank takes the
+        # same steps in the same order).
+        for ci, case in enumerate(CASES):
+            for layout in LAYOUTS:
+                B, Hq, Hkv, L, d, causal = case
+                w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
+                                    seed=11 + world + ci)
+                q, k, v = (x.double() for x in workloads.make_qkv(w))
+                bs, fin, init = _oracle_compute()
+                qc, kc, vc = (shard(x, rank, world, layout) for x in (q, k, v))
+                before = [x.clone() for x in (qc, kc, vc)]
+                out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, layout=layout, block_step=bs,
+                                          finalize=fin, init_state=init)
+                # The ring only reads the caller's chunks.
+                assert all(torch.equal(a, b) for a, b in zip(before, (qc, kc, vc)))
+                ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
+                ro = shard(torch.from_numpy(ro), rank, world, layout).numpy()
+                rl = shard(torch.from_numpy(rl), rank, world, layout, dim=2).numpy()
+                results[(rank, ci, layout)] = (float(np.max(np.abs(out.numpy() - ro))),
+                                               float(np.max(np.abs(lse.numpy() - rl))))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3, 4])
-@pytest.mark.parametrize("case", [(1, 2, 2, 16, 8, True), (2, 4, 2, 12, 8, False), (1, 4, 1, 9, 4, True)])
-def test_ring_protocol_matches_full_attention(world, case):
+def _run_ranks(target, world):
     ctx = mp.get_context("spawn")
-    mgr = ctx.Manager()
-    results = mgr.dict()
+    results = ctx.Manager().dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, case, results)) for r in range(world)]
+    procs = [ctx.Process(target=target, args=(r, world, port, results)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
-        p.join(timeout=120)
+        p.join(timeout=300)
         assert p.exitcode == 0, f"rank exited with {p.exitcode}"
-    assert sorted(results.keys()) == list(range(world))
-    for r, (eo, el) in results.items():
-        assert eo <= 1e-10 and el <= 1e-10, (r, eo, el)
+    got = dict(results)
+    assert sorted(got) == sorted((r, ci, lay) for r in range(world) for ci in range(len(CASES)) for lay in LAYOUTS)
+    return got
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_ring_protocol_matches_full_attention(world):
+    for key, (eo, el) in _run_ranks(_worker, world).items():
+        assert eo <= 1e-10 and el <= 1e-10, (key, eo, el)
 
 
 def _oracle_bwd_step():
@@ -109,52 +123,44 @@ def _oracle_bwd_step():
 
     return block_step_bwd
 
+def _add_and_clear_cpu(acc, part):
+    acc += part
+    part.zero_()
 
-def _bwd_worker(rank, world, port, case, results):
-    import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    sys.path.insert(0, root)
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+
+def _bwd_worker(rank, world, port, results):
+    _setup(rank, world, port)
     try:
         import oracle
         import workloads
-        from long_context_exact_blockwise_b200.ring import ring_attention_bwd
+        from long_context_exact_blockwise_b200.ring import ring_attention_bwd, shard
 
-        B, Hq, Hkv, L, d, causal = case
-        w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
-                            seed=31 + world)
-        q, k, v = (x.double() for x in workloads.make_qkv(w))
-        dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5), dtype=torch.float64)
-        out, lse = (torch.from_numpy(x) for x in oracle.attention_ref(q, k, v, causal=causal, scale=w.scale))
-        sl = slice(rank * L, (rank + 1) * L)
-        chunks = [x[:, sl].contiguous() for x in (q, k, v, out, dout)]
-        before = [x.clone() for x in chunks]
-        dq, dk, dv = ring_attention_bwd(*chunks, lse[:, :, sl].contiguous(), causal=causal, scale=w.scale,
-                                        block_step_bwd=_oracle_bwd_step())
-        assert all(torch.equal(a, b) for a, b in zip(before, chunks))
-        rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=causal, scale=w.scale)
-        results[rank] = tuple(float(np.max(np.abs(g.numpy() - r[:, sl]))) for g, r in ((dq, rq), (dk, rk), (dv, rv)))
+        for ci, case in enumerate(CASES):
+            for layout in LAYOUTS:
+                B, Hq, Hkv, L, d, causal = case
+                w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
+                                    seed=31 + world + ci)
+                q, k, v = (x.double() for x in workloads.make_qkv(w))
+                dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5), dtype=torch.float64)
+                out, lse = (torch.from_numpy(x) for x in oracle.attention_ref(q, k, v, causal=causal, scale=w.scale))
+                chunks = [shard(x, rank, world, layout) for x in (q, k, v, out, dout)]
+                before = [x.clone() for x in chunks]
+                dq, dk, dv = ring_attention_bwd(*chunks, shard(lse, rank, world, layout, dim=2), causal=causal,
+                                                scale=w.scale, layout=layout, block_step_bwd=_oracle_bwd_step(),
+                                                add_and_clear=_add_and_clear_cpu)
+                assert all(torch.equal(a, b) for a, b in zip(before, chunks))
+                rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=causal, scale=w.scale)
+                results[(rank, ci, layout)] = tuple(
+                    float(np.max(np.abs(g.numpy() - shard(torch.from_numpy(r), rank, world, layout).numpy())))
+                    for g, r in ((dq, rq), (dk, rk), (dv, rv)))
     finally:
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 3, 4])
-@pytest.mark.parametrize("case", [(1, 2, 2, 16, 8, True), (2, 4, 2, 12, 8, False), (1, 4, 1, 9, 4, True)])
-def test_ring_backward_protocol_matches_full_gradient(world, case):
-    ctx = mp.get_context("spawn")
-    results = ctx.Manager().dict()
-    port = _free_port()
-    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, case, results)) for r in range(world)]
-    for p in procs:
-        p.start()
-    for p in procs:
-        p.join(timeout=120)
-        assert p.exitcode == 0, f"rank exited with {p.exitcode}"
-    assert sorted(results.keys()) == list(range(world))
-    for r, errs in results.items():
-        assert max(errs) <= 1e-10, (r, errs)
+def test_ring_backward_protocol_matches_full_gradient(world):
+    for key, errs in _run_ranks(_bwd_worker, world).items():
+        assert max(errs) <= 1e-10, (key, errs)
 
 
 def test_ring_visit_order_matches_schedule_figure():
@@ -198,3 +204,36 @@ def test_ring_peer_loss_surfaces_as_error():
         p.join(timeout=120)
     assert all(p.exitcode is not None for p in procs), "a rank hung"
     assert results.get(0, "").startswith("error"), dict(results)
+
+
+def test_zigzag_layout_balances_causal_work():
+    # Causal visits that are not skipped, per rank: the contiguous layout
+    # gives rank i (i + 1) of them; the zigzag layout gives every rank the same
+    # number of (query piece, key piece) pairs with work in them.
+    from long_context_exact_blockwise_b200.ring import chunk_ids, ring_visit_order
+
+    def work(rank, world, layout):
+        n = len(chunk_ids(rank, world, layout))
+        pairs = 0
+        for owner in ring_visit_order(rank, world):
+            for kc in chunk_ids(owner, world, layout):
+                for qc in chunk_ids(rank, world, layout):
+                    pairs += 2 if kc < qc else (1 if kc == qc else 0)  # full tile = 2 halves, diagonal = 1
+        return pairs / n ** 2
+
+    for world in (2, 3, 4, 8):
+        contiguous = [work(r, world, "contiguous") for r in range(world)]
+        zigzag = [work(r, world, "zigzag") for r in range(world)]
+        assert contiguous == [2 * r + 1 for r in range(world)]
+        assert len(set(zigzag)) == 1, zigzag
+        assert sum(zigzag) == sum(contiguous)
+
+
+def test_shard_layouts_partition_the_sequence():
+    from long_context_exact_blockwise_b200.ring import shard
+    x = torch.arange(24).reshape(1, 24, 1, 1)
+    for layout in ("contiguous", "zigzag"):
+        got = torch.cat([shard(x, r, 3, layout) for r in range(3)], dim=1).flatten().tolist()
+        assert sorted(got) == list(range(24))
+    assert shard(x, 0, 3, "zigzag").flatten().tolist() == [0, 1, 2, 3, 20, 21, 22, 23]
+    assert shard(x, 1, 3, "zigzag").flatten().tolist() == [4, 5, 6, 7, 16, 17, 18, 19]
