@@ -1169,6 +1169,7 @@ cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t st) {
   if (a.B <= 0 || a.N_q <= 0) return cudaSuccess;
   if (decode_rows(a, mode) > 0) return launch_decode_sm100(a, mode, st);
   const Sm100Geometry geo = sm100_geometry(a, mode);
+  if (geo.two && fwd2_applies(a, mode)) return launch_fwd2_sm100(a, mode, st);
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
   if (encode_map(&prm.tm_q, a.q, a.d, a.Hq, a.N_q, a.B, geo.gpack) != CUDA_SUCCESS)

@@ -60,6 +60,13 @@ struct ProblemArgs {
 // Tensor-core path (tcgen05 + TMEM + TMA), bf16 inputs, d in {64, 128}.
 cudaError_t launch_fwd_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
 
+// Pair (cta_group::2) kernel for long query blocks (d = 128, bf16, final or
+// split-KV output): whether it takes a problem, and its launcher.
+// launch_fwd_sm100 routes such problems to it when RINGATTN_PAIR=1 (off by
+// default: it measured slower than the single-CTA kernel).
+bool fwd2_applies(const ProblemArgs& a, int mode);
+cudaError_t launch_fwd2_sm100(const ProblemArgs& a, int mode, cudaStream_t stream);
+
 // Keys-on-M decode kernel (d = 128, incremental queries with G * N_q <= 32
 // rows per KV head): rows per block it would use (16 or 32; 0 = not
 // applicable), and its launcher.  launch_fwd_sm100 routes such problems to it.

@@ -16,6 +16,7 @@
 #include "fwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "decode_f8_sm100.cuh"
+#include "fwd2_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "fwd_simt.cuh"
 #include "merge.cuh"

@@ -18,8 +18,11 @@ from parity_util import TOL_LSE, TOL_OUT, ra
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("N", [128, 256])  # one query tile / two query tiles, one CTA
-def test_bounded_wait_expiry_reports_status_and_context_survives(monkeypatch, N):
+# One query tile; two query tiles in one CTA; the CTA-pair kernel (one and
+# two pair tiles).
+@pytest.mark.parametrize("N,pair", [(128, ""), (256, ""), (256, "1"), (600, "1")])
+def test_bounded_wait_expiry_reports_status_and_context_survives(monkeypatch, N, pair):
+    monkeypatch.setenv("RINGATTN_PAIR", pair)
     R = ra()
     w = workloads.small(B=1, Hq=1, Hkv=1, N_q=N, d=128, causal=True, P=1, seed=5)
     q, k, v = workloads.make_qkv(w, device="cuda")
