@@ -127,7 +127,7 @@ def kernel_name(w: workloads.Workload, bwd: bool) -> str:
         return "simt_attn_kernel"
     rows = (w.Hq // w.Hkv) * w.N_q
     if w.d == 128 and w.cache_idx > 0 and w.window < 0:
-        if w.kv_dtype == "fp8" and rows <= 16:
+        if w.kv_dtype == "fp8" and (rows <= 16 or (rows <= 32 and w.Hq // w.Hkv <= 16)):
             return "decode_f8_sm100_kernel (FP8 KV on the 8-bit MMA path)"
         if w.kv_dtype != "fp8" and rows <= 16:
             return "decode_sm100_kernel"

@@ -37,6 +37,8 @@
  *     is enqueued asynchronously on it; no call synchronises unless the
  *     environment variable RINGATTN_DEBUG=1 is set (then each call
  *     synchronises and also reports the device status word).
+ *   - RINGATTN_NVTX=1 wraps every compute entry point in an NVTX range named
+ *     after it, for profilers; with no profiler attached it does nothing.
  *   - Every call returns a ring_attn_status.  Arguments are validated on the
  *     host before anything is launched; an invalid call launches nothing.
  *     ring_attn_error_string() turns a status into text; after

@@ -238,18 +238,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16
       : "memory");
 }
 
-// Ties 32 registers to this point of the program: later uses read them
-// after everything issued before it (such as a tcgen05.wait::ld that
-// completes their load), and the compiler cannot move those uses earlier.
-__device__ __forceinline__ void reg_tie32(float (&r)[32]) {
-  asm volatile(""
-               : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]), "+f"(r[6]), "+f"(r[7]),
-                 "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]), "+f"(r[12]), "+f"(r[13]), "+f"(r[14]),
-                 "+f"(r[15]), "+f"(r[16]), "+f"(r[17]), "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]),
-                 "+f"(r[22]), "+f"(r[23]), "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]),
-                 "+f"(r[29]), "+f"(r[30]), "+f"(r[31]));
-}
-
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format, version 1):
 // start address, leading and stride byte offsets (all >> 4), 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {

@@ -637,14 +637,17 @@ cudaError_t launch_decode_f8_sm100(const DecParams& prm, int NR, int mode, long 
 // the keys-on-M decode kernels take: 16 or 32 (0: they do not apply).
 int decode_rows(const ProblemArgs& a, int mode) {
   if (mode == kModeState || a.d != kDecD || a.wa_period > 0 || a.q_pos0 <= 0) return 0;
-  // RINGATTN_DECODE: "0" never; "all" up to 32 rows; default up to 16 rows
-  // (at 32 rows the general kernel measured faster, for both cache types).
+  // RINGATTN_DECODE: "0" never; "all" up to 32 rows in one block; default up
+  // to 16 rows for a bf16 cache (at 32 rows the general kernel measured
+  // faster).  An FP8 cache takes up to 32 rows by default, as 16-row blocks
+  // (two CTAs per SM; the row blocks of one KV head share its tiles in L2).
   const char* ov = std::getenv("RINGATTN_DECODE");
   if (ov && ov[0] == '0') return 0;
   const bool all = ov && std::strcmp(ov, "all") == 0;
   const long long G = a.Hq / a.Hkv;
   const long long rows = G * a.N_q;
-  const int nr = rows <= 16 ? 16 : (rows <= 32 && all ? 32 : 0);
+  const bool f8_blocks = a.kv8 && RA_DEC8_NATIVE && !all && rows <= 32;
+  const int nr = (rows <= 16 || f8_blocks) ? 16 : (rows <= 32 && all ? 32 : 0);
   if (nr == 0 || G > nr || nr % G != 0) return 0;
   return nr;
 }

@@ -67,17 +67,6 @@ constexpr float kSlackSum = 256.f;
 #define RA_EXP2_POLY_MASK 0x00
 #endif
 constexpr int kExp2PolyMask = RA_EXP2_POLY_MASK;
-// Two-tile CTAs: load S in two halves and start the first half's
-// exponentials while the second half is still in flight (1), or load all of
-// S before the softmax starts (0).
-#ifndef RA_FWD_SPLIT_LD
-#define RA_FWD_SPLIT_LD 0
-#endif
-// Two-tile CTAs: publish P in two halves so PV on keys 0..63 starts while
-// the softmax finishes keys 64..127 (1), or publish P whole (0).
-#ifndef RA_FWD_SPLITPV2
-#define RA_FWD_SPLITPV2 0
-#endif
 // FP8-KV kernel ring depths at d = 128 (bf16 slots, FP8 slots).
 #ifndef RA_KV8_NSLOT
 #define RA_KV8_NSLOT 4
@@ -274,42 +263,11 @@ __device__ __forceinline__ bool tile_needs_mask(const QTile& q, int k0, int kend
 // float values.  Bit i of EMU set: pairs whose index is i mod 8 use
 // exp2_poly2 (FMA pipe) instead of ex2 (MUFU).  EMU is a compile-time
 // constant so each pair's choice is fixed in the generated code.
-#ifndef RA_SOFTMAX_PIPE
-#define RA_SOFTMAX_PIPE 0
-#endif
 template <int EMU, int H>
 __device__ __forceinline__ float softmax_p_half(const float (&s)[128], float sl, float base, uint32_t s_tmem) {
   const float2 sl2 = make_float2(sl, sl);
   const float2 nb2 = make_float2(-base, -base);
   float2 sum0 = make_float2(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
-#if RA_SOFTMAX_PIPE
-  if constexpr (EMU == 0) {
-    // Software-pipelined: the argument of pair i + 1 and the bf16 pack of
-    // pair i - 1 sit between the two exponentials of pair i in program order.
-    float2 acc[4] = {sum0, sum0, sum0, sum0};
-#pragma unroll
-    for (int c = 2 * H; c < 2 * H + 2; ++c) {
-      uint32_t u[16];
-      float2 a = __ffma2_rn(make_float2(s[c * 32], s[c * 32 + 1]), sl2, nb2);
-      float2 prev = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float2 an = a;
-        if (i + 1 < 16) an = __ffma2_rn(make_float2(s[c * 32 + 2 * i + 2], s[c * 32 + 2 * i + 3]), sl2, nb2);
-        const float ex = ex2(a.x);
-        if (i > 0) u[i - 1] = pack_bf16x2(prev.x, prev.y);
-        const float ey = ex2(a.y);
-        prev = make_float2(ex, ey);
-        acc[i & 3] = __fadd2_rn(acc[i & 3], prev);
-        a = an;
-      }
-      u[15] = pack_bf16x2(prev.x, prev.y);
-      tmem_st16(s_tmem + c * 16, u);
-    }
-    const float2 sa = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-    return sa.x + sa.y;
-  }
-#endif
 #pragma unroll
   for (int c = 2 * H; c < 2 * H + 2; ++c) {
     uint32_t u[16];
@@ -458,8 +416,7 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
   // rest of the softmax).  Two-tile CTAs ping-pong instead; the extra
   // signalling measured slower there.
   constexpr bool kSplitS = (NQT == 1);
-  constexpr bool kSplitPV = (NQT == 1) || (RA_FWD_SPLITPV2 != 0);
-  constexpr bool kSplitLd = (NQT == 2) && (RA_FWD_SPLIT_LD != 0);
+  constexpr bool kSplitPV = (NQT == 1);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -841,45 +798,20 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
         }
         tc_fence_after();
         float s[128];
-        // Keys 64..127 may still be in flight (kSplitLd): wait_hi() completes
-        // their load before any use.
-        bool hi_pending = false;
-        auto wait_hi = [&]() {
-          if (kSplitLd && hi_pending) {
-            tc_wait_ld();
-            reg_tie32(*reinterpret_cast<float(*)[32]>(&s[64]));
-            reg_tie32(*reinterpret_cast<float(*)[32]>(&s[96]));
-            hi_pending = false;
-          }
-        };
-        if constexpr (kSplitLd) {
-          tmem_ld32(s_tmem, *reinterpret_cast<float(*)[32]>(&s[0]));
-          tmem_ld32(s_tmem + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-          tc_wait_ld();
-          reg_tie32(*reinterpret_cast<float(*)[32]>(&s[0]));
-          reg_tie32(*reinterpret_cast<float(*)[32]>(&s[32]));
-          tmem_ld32(s_tmem + 64, *reinterpret_cast<float(*)[32]>(&s[64]));
-          tmem_ld32(s_tmem + 96, *reinterpret_cast<float(*)[32]>(&s[96]));
-          hi_pending = true;
-        } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float (&r)[32] = *reinterpret_cast<float(*)[32]>(&s[c * 32]);
-            tmem_ld32(s_tmem + c * 32, r);
-          }
-          tc_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          float (&r)[32] = *reinterpret_cast<float(*)[32]>(&s[c * 32]);
+          tmem_ld32(s_tmem + c * 32, r);
         }
+        tc_wait_ld();
         // S is in registers: the issuer may now overwrite its columns 64..127
         // with the next tile's scores (the first 64 columns get P).
         if constexpr (kSplitS) warp_arrive_after_tc(BAR_SC(t), lane);
-        const bool masked = tile_needs_mask<WA>(q, cur.k0, cur.kend, p.causal);
-        // Only the one-pass exponentials of an unmasked tile start before
-        // every score is in registers.
-        if (!fold || masked || n == 0) wait_hi();
         if (!fold) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] *= scale_l2;
         }
+        const bool masked = tile_needs_mask<WA>(q, cur.k0, cur.kend, p.causal);
         if (WA && masked) {
           // This row's window [pos - W, pos] and the CTA's anchors, inside
           // the keys of this tile (tile-relative).
@@ -921,7 +853,6 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
         // P is published.  A row's first tile, and single-tile CTAs (which
         // publish half of P early), take the max first.
         auto row_max = [&]() {
-          wait_hi();
           // Four independent chains of 3-input max.
           float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
@@ -943,7 +874,6 @@ __global__ void __launch_bounds__(128 + 128 * NQT + (NSLOT8 > 0 ? 128 : 0), 1)
             tc_wait_st();
             warp_arrive_after_tc(BAR_PA(t), lane);
           }
-          wait_hi();
           r += masked ? softmax_p_half<0, 1>(s, sl, base, s_tmem)
                       : softmax_p_half<kExp2PolyMask, 1>(s, sl, base, s_tmem);
           return r;

@@ -8,6 +8,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -74,6 +76,21 @@ int check_device(int* num_sms) {
 
 // After a launch: report launch errors; in debug mode also synchronise and
 // read the device status word.
+// RINGATTN_NVTX=1: every compute entry point is an NVTX range named after
+// it, for profilers.  NVTX here is header-only: without a profiler attached
+// the calls do nothing.
+struct NvtxScope {
+  bool on;
+  explicit NvtxScope(const char* name) : on(env_flag("RINGATTN_NVTX")) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxScope() {
+    if (on) nvtxRangePop();
+  }
+  NvtxScope(const NvtxScope&) = delete;
+  NvtxScope& operator=(const NvtxScope&) = delete;
+};
+
 int finish(cudaError_t e, cudaStream_t st, const char* where) {
   if (e != cudaSuccess) return set_cuda_error(e, where);
   if (env_flag("RINGATTN_DEBUG")) {
@@ -230,6 +247,7 @@ extern "C" {
 int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                   int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
                   void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd");
   int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
   if (r != RA_OK) return r;
   if (B == 0 || N_q == 0) return RA_OK;
@@ -250,6 +268,7 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
 int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
                                 int Hkv, int64_t N, int d, int64_t chunk, int P, int64_t window,
                                 int64_t anchor_period, float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_window_anchor");
   if (window < 0 || window > kMaxTokens || anchor_period <= 0 || anchor_period % 256 != 0 ||
       anchor_period > kMaxTokens)
     return RA_ERR_INVALID_ARG;
@@ -273,6 +292,7 @@ int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, voi
 int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const float* k_scale, const float* v_scale,
                         void* out, float* lse, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
                         int64_t chunk, int P, int64_t cache_idx, float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_fp8kv");
   if (!k_scale || !v_scale) return RA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u) return RA_ERR_INVALID_ARG;
   int r = validate_fwd(q, k8, v8, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
@@ -296,6 +316,7 @@ int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const flo
 int ring_attn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B, int Hq,
                       int Hkv, int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx,
                       float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_f32");
   int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, false);
   if (r != RA_OK) return r;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
@@ -318,6 +339,7 @@ int ring_attn_fwd_f32(const float* q, const float* k, const float* v, float* out
 int ring_attn_block_step(const void* q_chunk, const void* k_chunk, const void* v_chunk, int64_t q_off,
                          int64_t k_off, float* acc, float* m, float* l, int B, int Hq, int Hkv, int64_t Lq,
                          int64_t Lk, int d, int causal, float scale, int dtype, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_block_step");
   if (!q_chunk || !k_chunk || !v_chunk || !acc || !m || !l) return RA_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return RA_ERR_INVALID_ARG;
@@ -348,6 +370,7 @@ int ring_attn_block_step(const void* q_chunk, const void* k_chunk, const void* v
 
 int ring_attn_finalize(const float* acc, const float* m, const float* l, void* out, float* lse, int B, int Hq,
                        int64_t Lq, int d, int out_dtype, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_finalize");
   if (!acc || !m || !l || !out || !lse) return RA_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Lq < 0 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
   if (out_dtype != RA_DTYPE_BF16 && out_dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
@@ -362,6 +385,7 @@ int ring_attn_finalize(const float* acc, const float* m, const float* l, void* o
 
 int lse_merge(const float* o_parts, const float* lse_parts, int S, void* out, float* lse, int B, int Hq,
               int64_t N_q, int d, int out_dtype, void* stream) {
+  NvtxScope nvtx_scope("lse_merge");
   if (!o_parts || !lse_parts || !out || !lse) return RA_ERR_INVALID_ARG;
   if (S < 1 || B < 0 || Hq < 1 || N_q < 0 || (d != 64 && d != 128)) return RA_ERR_INVALID_ARG;
   if (out_dtype != RA_DTYPE_BF16 && out_dtype != RA_DTYPE_F32) return RA_ERR_INVALID_ARG;
@@ -409,6 +433,7 @@ extern "C" {
 int ring_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
                   int64_t cache_idx, float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_bwd");
   if (!dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
   if (!(aligned16(dout) && aligned16(dq) && aligned16(dk) && aligned16(dv))) return RA_ERR_INVALID_ARG;
   // Same shape rules as ring_attn_fwd (one chunk spanning the sequence).
@@ -433,6 +458,7 @@ int ring_attn_bwd_block_step(const void* q_chunk, const void* k_chunk, const voi
                              const void* dout_chunk, const float* lse_chunk, int64_t q_off, int64_t k_off,
                              float* dq_acc, float* dk_acc, float* dv_acc, int B, int Hq, int Hkv, int64_t Lq,
                              int64_t Lk, int d, int causal, float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_bwd_block_step");
   if (!q_chunk || !k_chunk || !v_chunk || !out_chunk || !dout_chunk || !lse_chunk) return RA_ERR_INVALID_ARG;
   if (!dq_acc || !dk_acc || !dv_acc) return RA_ERR_INVALID_ARG;
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
@@ -462,6 +488,7 @@ int ring_attn_bwd_block_step(const void* q_chunk, const void* k_chunk, const voi
 }
 
 int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_exp2_poly");
   if (!x || !y || n < 0) return RA_ERR_INVALID_ARG;
   if (n == 0) return RA_OK;
   int r = check_device(nullptr);
@@ -471,6 +498,7 @@ int ring_attn_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
 }
 
 int ring_attn_add_and_clear(float* acc, float* part, int64_t n, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_add_and_clear");
   if (n < 0) return RA_ERR_INVALID_ARG;
   if (n == 0) return RA_OK;
   if (!acc || !part || acc == part) return RA_ERR_INVALID_ARG;
@@ -530,6 +558,7 @@ int noalloc_scratch_address(void** out) {
 extern "C" int ring_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                                      int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk,
                                      int P, int64_t cache_idx, float scale, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_noalloc");
   int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
   if (r != RA_OK) return r;
   if (cache_idx < 0) {

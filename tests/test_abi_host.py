@@ -171,3 +171,14 @@ def test_add_and_clear_validation():
     assert L.ring_attn_add_and_clear(None, FAKE, 8, None) == ra.RA_ERR_INVALID_ARG
     assert L.ring_attn_add_and_clear(FAKE, FAKE, 8, None) == ra.RA_ERR_INVALID_ARG  # the same buffer twice
     assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20002), 8, None) == ra.RA_ERR_INVALID_ARG  # unaligned
+
+
+def test_nvtx_ranges_switch_keeps_validation(monkeypatch):
+    # RINGATTN_NVTX=1 wraps every compute entry point in an NVTX range; with
+    # no profiler attached the ranges do nothing and validation is unchanged.
+    ra = _lib()
+    monkeypatch.setenv("RINGATTN_NVTX", "1")
+    L = ra.lib
+    assert L.ring_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 128, 128, 96, 1, 128, 1, -1, 0.1, None) == \
+        ra.RA_ERR_INVALID_ARG
+    assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20000), 0, None) == ra.RA_OK
