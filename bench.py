@@ -53,19 +53,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.829857 GB read + 0.254630 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.084487e9, "src": "25f212287f8997c7"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073930 GB read + 0.004202 GB written.
-    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078132e9, "src": "7ee2ab864cd3d8e7"},
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.828320 GB read + 0.253901 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.082221056e9, "src": "4e9287c179a0d8d2"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073936 GB read + 0.004240 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078175488e9, "src": "fa8b792e8808ecd6"},
     # The full-length decodes scale the quarter-length captures by their 4x KV
     # length (traffic is K/V streaming, proportional to N_kv).
-    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078132e9, "src": "7ee2ab864cd3d8e7"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537044 GB read + 0.004457 GB written.
-    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541501e9, "src": "7ee2ab864cd3d8e7"},
-    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541501e9, "src": "7ee2ab864cd3d8e7"},
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078175488e9, "src": "fa8b792e8808ecd6"},
+    # profiles/decode_f8_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537039 GB read + 0.004585 GB written.
+    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541623808e9, "src": "fa8b792e8808ecd6"},
+    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541623808e9, "src": "fa8b792e8808ecd6"},
     # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step (prep + dK/dV + dQ):
-    # 0.541 + 0.010, 1.084 + 0.508, 1.085 + 0.256 GB read + written.
-    "llama7b_prefill_N32768 bwd": {"bytes": 3.485068e9, "src": "6dd983a4b4a81d8e"},
+    # 0.541 + 0.011, 1.085 + 0.505, 1.084 + 0.252 GB read + written.
+    "llama7b_prefill_N32768 bwd": {"bytes": 3.477207552e9, "src": "ae663e30030606ff"},
 }
 
 
@@ -74,8 +74,9 @@ NCU_TRAFFIC = {
 # decode kernel, which shares the FP8 converter and cursor code of the
 # forward's sources) and "bwd".
 _NOT_IN_HASH = {"fwd": {"bwd_sm100.cuh", "decode_sm100.cuh", "decode_f8_sm100.cuh"},
-                "decode": {"bwd_sm100.cuh", "fwd_simt.cuh"},
-                "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh", "decode_f8_sm100.cuh"}}
+                "decode": {"bwd_sm100.cuh", "fwd_simt.cuh", "fwd2_sm100.cuh"},
+                "bwd": {"fwd_sm100.cuh", "fwd_simt.cuh", "merge.cuh", "decode_sm100.cuh", "decode_f8_sm100.cuh",
+                        "fwd2_sm100.cuh"}}
 
 
 def kernel_source_hash(pass_: str = "fwd") -> str:

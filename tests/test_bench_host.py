@@ -39,6 +39,9 @@ def test_backward_hash_ignores_forward_and_decode_kernels():
     assert "decode_sm100.cuh" in bench._NOT_IN_HASH["bwd"]
     assert "bwd_sm100.cuh" in bench._NOT_IN_HASH["fwd"]
     assert "bwd_sm100.cuh" in bench._NOT_IN_HASH["decode"]
+    # The CTA-pair forward kernel changes neither the decode nor the backward kernels.
+    assert "fwd2_sm100.cuh" in bench._NOT_IN_HASH["decode"]
+    assert "fwd2_sm100.cuh" in bench._NOT_IN_HASH["bwd"]
 
 
 def test_traffic_entries_name_known_workloads():
