@@ -123,6 +123,19 @@ __device__ __forceinline__ void mma_tmem_x_tile(uint32_t d_tmem, uint32_t a_tmem
     umma_ts(d_tmem, a_tmem + EwSplit<EW>::packed_col(kk), bd + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// D(tmem, M=128 x N=D) (+)= A(smem, 128 x 128, K-major in two 64-column
+// blocks) B(128 rows x D, MN-major).
+template <int D>
+__device__ __forceinline__ void mma_rows_x_rows_mn(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBT, D, 1);
+  const uint64_t ad = kmajor_desc(a_addr), bd = mnmajor_desc(b_addr);
+#pragma unroll
+  for (int kk = 0; kk < kBT / 16; ++kk) {
+    const uint32_t aoff = (kk / 4) * (kBT * 128) + (kk % 4) * 32;
+    umma_ss(d_tmem, ad + (aoff >> 4), bd + ((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int D, int head, int row,
                                          int b) {
   for (int hf = 0; hf < D / 64; ++hf) tma_load_4d(dst + hf * (kBT * 128), map, bar, hf * 64, head, row, b);
@@ -160,14 +173,21 @@ struct DkdvLayout {
   static constexpr int kTile = kBT * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
-  static constexpr int kStage0 = kV + kTile;                 // per stage: Q, dout, lse2[128], D[128]
+  static constexpr int kStage0 = kV + kTile;  // per stage: Q, dout, lse2[128], D[128]
   static constexpr int kStageBytes = 2 * kTile + 2 * kBT * 4;
-  static constexpr int kBars = kStage0 + 2 * kStageBytes;  // kv_full, qf[2], qe[2], s, p, done, drain, dp, ds
-  static constexpr int kMisc = kBars + 12 * 8;
+  // P^T as bf16, the A operand of dV += P^T dout: 128 key rows x 128 query
+  // columns, K-major, two 64-column blocks with the 128-byte swizzle.
+  static constexpr int kP = kStage0 + 2 * kStageBytes;
+  static constexpr int kBars = kP + kBT * kBT * 2;  // kv_full, qf[2], qe[2], s, p, done, drain, dp, ds, sfree, pfree
+  static constexpr int kMisc = kBars + 13 * 8;
   static constexpr int kBytes = kMisc + 16;
-  // More than half the SM's shared memory: one CTA per SM, so the 512-column
-  // TMEM allocation never waits on another CTA.
-  static constexpr int kAlloc = kBytes + 1024 < 120 * 1024 ? 120 * 1024 : kBytes + 1024;
+  // The tiles need 1024-byte alignment.  At D = 128 the layout leaves room
+  // for 896 bytes of padding only, so the kernel requires a dynamic
+  // shared-memory base aligned to 128 bytes (it checks, and reports
+  // RA_ERR_UNSUPPORTED otherwise).  More than half the SM's shared memory:
+  // one CTA per SM, so the 512-column TMEM allocation never waits.
+  static constexpr int kSlack = 1024 - 128;
+  static constexpr int kAlloc = kBytes + kSlack < 120 * 1024 ? 120 * 1024 : kBytes + kSlack;
 };
 
 template <int D>
@@ -175,6 +195,10 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
   using L = DkdvLayout<D>;
   constexpr int kEw = kEwDkdv, kNH = EwSplit<kEw>::kNH, kCW = EwSplit<kEw>::kCW;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 127u) {  // see DkdvLayout::kSlack
+    if (threadIdx.x == 0) atomicExch(&g_status, (int)RA_ERR_UNSUPPORTED);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kBars;
@@ -182,7 +206,8 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
   auto BAR_QF = [&](int s) { return bar0 + 8u * (1 + s); };
   auto BAR_QE = [&](int s) { return bar0 + 8u * (3 + s); };
   const uint32_t BAR_S = bar0 + 8u * 5, BAR_P = bar0 + 8u * 6, BAR_DONE = bar0 + 8u * 7, BAR_DRAIN = bar0 + 8u * 8;
-  const uint32_t BAR_DP = bar0 + 8u * 9, BAR_DS = bar0 + 8u * 10;
+  const uint32_t BAR_DP = bar0 + 8u * 9, BAR_DS = bar0 + 8u * 10, BAR_SFREE = bar0 + 8u * 11;
+  const uint32_t BAR_PFREE = bar0 + 8u * 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   auto stage_q = [&](int s) { return sbase + L::kStage0 + s * L::kStageBytes; };
@@ -222,6 +247,8 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
     mbar_init(BAR_DRAIN, 1);
     mbar_init(BAR_DP, 1);
     mbar_init(BAR_DS, kEw);
+    mbar_init(BAR_SFREE, kEw);
+    mbar_init(BAR_PFREE, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -270,12 +297,12 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
   } else if (warp == 1) {
     if (lane == 0) {
       // Software pipeline over iterations w (one query tile of one head):
-      //   dV_w += P^T_w dout_w  |  S^T_{w+1}  |  dK_w += dS^T_w Q_w  |  dP^T_{w+1}
-      // so the tensor pipe works on the next tile's S^T while the
-      // elementwise warps form dS^T_w, and on dK_w / dP^T_{w+1} while they
-      // form P^T_{w+1}.  S^T_{w+1} overwrites the columns dV_w reads P^T_w
-      // from, and dP^T_{w+1} those dK_w reads dS^T_w from: tcgen05 MMAs of
-      // one thread run in issue order.  Each S / dP commit comes after the
+      //   S^T_{w+1}, dV_w += P^T_w dout_w  |  dK_w += dS^T_w Q_w  |  dP^T_{w+1}
+      // P^T goes to shared memory, so S^T_{w+1} may overwrite S^T_w as soon
+      // as the elementwise warps hold S^T_w in registers (SFREE): the tensor
+      // pipe computes the next scores while they form P^T_w.  dP^T_{w+1}
+      // overwrites the columns dK_w reads dS^T_w from: tcgen05 MMAs of one
+      // thread run in issue order.  Each S / dP commit comes after the
       // elementwise warps have passed the previous wait on the same barrier,
       // so no barrier runs two phases ahead of its waiters.
       bool ok = mbar_wait(BAR_KV, 0, abort_flag);
@@ -290,15 +317,39 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
       for (int w = 0; w < n_work && ok; ++w) {
         const int s = w & 1;
         const bool more = w + 1 < n_work;
-        if (!(ok = mbar_wait(BAR_P, w & 1, abort_flag))) break;
-        tc_fence_after();
-        mma_tmem_x_tile<D, kEw>(T_DV, T_ST, stage_do(s), w > 0);   // dV += P^T dout
-        if (more) {
-          if (!(ok = mbar_wait(BAR_QF(s ^ 1), ((w + 1) >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          mma_rows_x_rows<D>(T_ST, sbase + L::kK, stage_q(s ^ 1));
-          tc_commit(BAR_S);
+        // S^T_{w+1} (once the warps hold S^T_w and Q_{w+1} has landed) and
+        // dV_w (once P^T_w is written) go out in the order their inputs
+        // arrive, S^T first when both are ready: a late Q tile must not hold
+        // up dV_w, whose completion frees the P^T buffer.
+        if (more && !(ok = mbar_wait(BAR_SFREE, w & 1, abort_flag))) break;
+        bool s_todo = more, v_todo = true;
+        const uint32_t qpar = ((w + 1) >> 1) & 1;
+        const unsigned long long t0 = globaltimer_ns();
+        for (uint32_t i = 1; s_todo || v_todo; ++i) {
+          if (s_todo && mbar_test(BAR_QF(s ^ 1), qpar)) {
+            tc_fence_after();
+            mma_rows_x_rows<D>(T_ST, sbase + L::kK, stage_q(s ^ 1));  // S^T_{w+1}
+            tc_commit(BAR_S);
+            s_todo = false;
+          } else if (v_todo && mbar_test(BAR_P, w & 1)) {
+            tc_fence_after();
+            mma_rows_x_rows_mn<D>(T_DV, sbase + L::kP, stage_do(s), w > 0);  // dV += P^T dout
+            tc_commit(BAR_PFREE);
+            v_todo = false;
+          } else if ((i & 255u) == 0u) {
+            if (*abort_flag) {
+              ok = false;
+              break;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              atomicExch(&g_status, (int)RA_ERR_DEVICE_TIMEOUT);
+              ok = false;
+              break;
+            }
+          }
         }
+        if (!ok) break;
         if (!(ok = mbar_wait(BAR_DS, w & 1, abort_flag))) break;
         tc_fence_after();
         mma_tmem_x_tile<D, kEw>(T_DK, T_DPT, stage_q(s), w > 0);   // dK += dS^T Q
@@ -322,6 +373,8 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
     const uint32_t lb = lq + (uint32_t)g0;
     const long long key = (long long)j0 + r;
     const float sl = p.scale_log2;
+    // This thread's row of the P^T buffer (K-major, 128-byte swizzle).
+    uint8_t* prow = smem + L::kP + r * 128;
     bool ok = true;
     for (int w = 0; w < n_work; ++w) {
       const int s = w & 1;
@@ -332,45 +385,59 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
       // (already complete) so the loads below observe the copied data.
       if (!(ok = mbar_wait(BAR_QF(s), (w >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      const float* lse2 = stage_lse(s);
-      const float* dD = stage_d(s);
+      const float* lse2 = stage_lse(s) + g0;
+      const float* dD = stage_d(s) + g0;
       // Causal: query column c is visible to this key iff
       // q_pos0 + qt*128 + c >= k_pos0 + key, i.e. c >= cmin.
       long long cm = p.causal ? (key + p.k_pos0 - p.q_pos0) - (long long)qt * kBT : -1;
       const int cmin = (int)(cm < 0 ? 0 : (cm > kBT ? kBT : cm));
-      // Phase 1: P^T (kept in registers for phase 2), bf16 over S^T.
+      // Phase 1: P^T (kept in registers for phase 2), bf16 to shared memory.
+      // The first 32 columns' exponentials overlap the load of the rest.
       float pv[kCW];
-#pragma unroll
-      for (int c = 0; c < kCW / 32; ++c) tmem_ld32(T_ST + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
+      tmem_ld32(T_ST + lb, *reinterpret_cast<float(*)[32]>(pv));
       tc_wait_ld();
+#pragma unroll
+      for (int c = 1; c < kCW / 32; ++c) tmem_ld32(T_ST + lb + c * 32, *reinterpret_cast<float(*)[32]>(pv + c * 32));
       // Only warps on the causal diagonal mask columns; the others skip the
       // selects (a warp-uniform choice, so no lanes diverge).
-      auto p_chunks = [&](auto masked) {
+      const bool diag = __any_sync(0xffffffffu, cmin > g0);
+      auto exps = [&](auto lo_c, auto hi_c, auto masked) {
 #pragma unroll
-        for (int c = 0; c < kCW / 32; ++c) {
-          uint32_t up[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int l0 = c * 32 + i, q0 = g0 + l0;
-            float p0 = ex2(fmaf(pv[l0], sl, -lse2[q0]));
-            float p1 = ex2(fmaf(pv[l0 + 1], sl, -lse2[q0 + 1]));
-            if constexpr (decltype(masked)::value) {
-              if (q0 < cmin) p0 = 0.f;
-              if (q0 + 1 < cmin) p1 = 0.f;
-            }
-            pv[l0] = p0;
-            pv[l0 + 1] = p1;
-            up[i / 2] = pack_bf16x2(p0, p1);
+        for (int l = decltype(lo_c)::value * 32; l < decltype(hi_c)::value * 32; ++l) {
+          float e = ex2(fmaf(pv[l], sl, -lse2[l]));
+          if constexpr (decltype(masked)::value) {
+            if (g0 + l < cmin) e = 0.f;
           }
-          tmem_st16(T_ST + lb + c * 16, up);
+          pv[l] = e;
         }
       };
-      if (__any_sync(0xffffffffu, cmin > g0))
-        p_chunks(std::true_type{});
+      using C0 = std::integral_constant<int, 0>;
+      using C1 = std::integral_constant<int, 1>;
+      using CN = std::integral_constant<int, kCW / 32>;
+      if (diag)
+        exps(C0{}, C1{}, std::true_type{});
       else
-        p_chunks(std::false_type{});
-      tc_wait_st();
+        exps(C0{}, C1{}, std::false_type{});
+      tc_wait_ld();
+      // S^T_w is in registers: the next tile's scores may overwrite it.
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR_SFREE);
+      if (diag)
+        exps(C1{}, CN{}, std::true_type{});
+      else
+        exps(C1{}, CN{}, std::false_type{});
+      // dV_{w-1} must have read the buffer before it is overwritten.
+      if (w > 0 && !(ok = mbar_wait(BAR_PFREE, (w - 1) & 1, abort_flag))) break;
+#pragma unroll
+      for (int c = 0; c < kCW / 8; ++c) {
+        // 8 query columns = one 16-byte chunk of the row's 64-column block.
+        const int q8 = (g0 + c * 8) >> 3;
+        *reinterpret_cast<uint4*>(prow + (q8 >> 3) * (kBT * 128) + (((q8 & 7) ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16x2(pv[c * 8], pv[c * 8 + 1]), pack_bf16x2(pv[c * 8 + 2], pv[c * 8 + 3]),
+                       pack_bf16x2(pv[c * 8 + 4], pv[c * 8 + 5]), pack_bf16x2(pv[c * 8 + 6], pv[c * 8 + 7]));
+      }
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR_P);
       // Phase 2: dS^T = P^T (dP^T - D), bf16 over dP^T.
@@ -384,8 +451,8 @@ __global__ void __launch_bounds__(EwSplit<kEwDkdv>::kThreads, 1) bwd_dkdv_kernel
         uint32_t uds[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const int l0 = c * 32 + i, q0 = g0 + l0;
-          uds[i / 2] = pack_bf16x2(pv[l0] * (dpt[i] - dD[q0]), pv[l0 + 1] * (dpt[i + 1] - dD[q0 + 1]));
+          const int l0 = c * 32 + i;
+          uds[i / 2] = pack_bf16x2(pv[l0] * (dpt[i] - dD[l0]), pv[l0 + 1] * (dpt[i + 1] - dD[l0 + 1]));
         }
         tmem_st16(T_DPT + lb + c * 16, uds);
       }

@@ -128,21 +128,46 @@ int validate_fwd(const void* q, const void* k, const void* v, const void* out, c
   return RA_OK;
 }
 
-// Number of KV splits for an incremental query: enough CTAs to keep every SM
-// busy for several waves.  RINGATTN_SPLITS overrides.
+// Number of KV splits for an incremental query (`items` CTAs per split, one
+// CTA per SM at a time).  RINGATTN_SPLITS overrides.
+//   - Decode shapes (at most 64 query rows) stream the KV cache: enough
+//     splits for about eight waves of CTAs in flight.
+//   - Otherwise every CTA does about the same work (whole ring steps of one
+//     query block), so the kernel takes (waves) x (ring steps per CTA).  The
+//     count minimising that, with a quarter step of per-CTA overhead, wins;
+//     ties go to fewer splits (fewer partials to write and merge).  512
+//     queries over 64 steps in 256 CTAs per split: 4 splits (1024 CTAs, 7
+//     waves of 16 steps) instead of 2 (512 CTAs, 4 waves of 32 steps, the
+//     last wave less than half full).
 int choose_splits(long long items, int P, int num_sms, long long n_q) {
   const char* ov = std::getenv("RINGATTN_SPLITS");
   if (ov && ov[0]) {
     int s = std::atoi(ov);
     return s < 1 ? 1 : (s > P ? P : s);
   }
-  const long long waves = n_q <= 64 ? 8 : 2;  // decode shapes stream KV: want many CTAs in flight
-  long long s = (waves * num_sms + items - 1) / items;
-  if (s < 1) s = 1;
-  if (s > P) s = P;
-  // Whole ring steps per split.
-  const int sps = (int)((P + s - 1) / s);
-  return (P + sps - 1) / sps;
+  if (items < 1) items = 1;
+  if (n_q <= 64) {
+    long long s = (8LL * num_sms + items - 1) / items;
+    if (s < 1) s = 1;
+    if (s > P) s = P;
+    // Whole ring steps per split.
+    const int sps = (int)((P + s - 1) / s);
+    return (P + sps - 1) / sps;
+  }
+  constexpr int kMaxSplits = 32;
+  int best = 1;
+  double best_cost = 0.0;
+  for (int sps = P; sps >= 1; --sps) {
+    const int s = (P + sps - 1) / sps;
+    if (s > kMaxSplits) break;
+    const long long waves = (items * s + num_sms - 1) / num_sms;
+    const double cost = (double)waves * (sps + 0.25);
+    if (sps == P || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 }  // namespace
