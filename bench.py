@@ -377,8 +377,9 @@ def run_ring(args, w, rank, world, device):
 
     The workload's whole sequence is cut into 2 * world chunks; rank i holds
     chunks i and 2 world - 1 - i (zigzag layout, equal causal work per rank)
-    and exchanges KV with its ring neighbours every step.  Total work is
-    fixed as world grows (strong scaling).  Returns the timing record.
+    and exchanges KV with its ring neighbours every step (one way, or with
+    --bidirectional each of its two chunks in its own direction).  Total work
+    is fixed as world grows (strong scaling).  Returns the timing record.
     """
     from long_context_exact_blockwise_b200 import ring
     import long_context_exact_blockwise_b200.ringattn as R
@@ -390,7 +391,8 @@ def run_ring(args, w, rank, world, device):
     del q, k, v
 
     def step():
-        return ring.ring_attention(qc, kc, vc, causal=w.causal, scale=w.scale, layout="zigzag")
+        return ring.ring_attention(qc, kc, vc, causal=w.causal, scale=w.scale, layout="zigzag",
+                                   bidirectional=args.bidirectional)
 
     for _ in range(args.warmup):
         step()
@@ -585,10 +587,15 @@ def main():
     ap.add_argument("--ring", action="store_true",
                     help="time ring.ring_attention across the N ranks (sequence-parallel ring, zigzag chunks, "
                          "strong scaling) instead of data-parallel replicas of the single-GPU kernel")
+    ap.add_argument("--bidirectional", action="store_true",
+                    help="with --ring: the bidirectional ring (each rank's two chunks travel in opposite "
+                         "directions)")
     ap.add_argument("--decode", default="5d1,5d1f8",
                     help="decode workloads timed after the forward prefill of config 2 and reported in the "
                          "line's 'decode' list (comma-separated keys; 'none' to skip)")
     args = ap.parse_args()
+    if args.bidirectional and not args.ring:
+        ap.error("--bidirectional needs --ring")
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
 
@@ -672,7 +679,8 @@ def main():
         res = run_ring(args, w, rank, world, device)
         ms_step = res["ms_total"] / args.steps
         value = flops / (ms_step * 1e-3) / 1e12
-        config["parallelism"] = f"sequence-parallel ring x{world} (zigzag chunks)"
+        config["parallelism"] = (f"sequence-parallel {'bidirectional ' if args.bidirectional else ''}ring x{world} "
+                                 "(zigzag chunks)")
         config["global_batch"] = w.B
         line = {"metric": "attention fwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,

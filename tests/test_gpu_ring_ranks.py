@@ -7,7 +7,8 @@ chunks, while the KV chunks and the travelling dK / dV accumulators move
 between the ranks as CPU tensors over gloo.  The kernels of different ranks
 never wait on one another.  Every rank's forward (out, lse) and backward
 (dq, dk, dv) must match the float64 oracle on its rows, for the contiguous
-and the zigzag chunk layouts, causal and not.
+and the zigzag chunk layouts, the one-way and the bidirectional ring, causal
+and not.
 """
 import os
 import socket
@@ -24,7 +25,8 @@ CASES = [  # (B, Hq, Hkv, L per rank, d, causal)
     (1, 4, 2, 256, 128, True),
     (2, 2, 2, 192, 64, False),
 ]
-LAYOUTS = ["contiguous", "zigzag"]
+# (chunk layout, bidirectional)
+MODES = [("contiguous", False), ("zigzag", False), ("contiguous", True), ("zigzag", True)]
 
 
 def _free_port():
@@ -83,16 +85,17 @@ def _worker(rank, world, port, results):
         dev = torch.device("cuda", 0)
         bs, fin, init, bs_bwd, add_clear = _cuda_compute(dev)
         for ci, (B, Hq, Hkv, L, d, causal) in enumerate(CASES):
-            for layout in LAYOUTS:
+            for layout, bi in MODES:
                 w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, causal=causal, P=world,
                                     seed=70 + 10 * world + ci)
                 q, k, v = workloads.make_qkv(w)  # bf16 on the CPU, the same on every rank
                 dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(71 + ci)).to(torch.bfloat16)
                 qc, kc, vc, dc = (shard(x, rank, world, layout) for x in (q, k, v, dout))
-                out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, layout=layout, block_step=bs,
-                                          finalize=fin, init_state=init)
+                out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, layout=layout, bidirectional=bi,
+                                          block_step=bs, finalize=fin, init_state=init)
                 dq, dk, dv = ring_attention_bwd(qc, kc, vc, out, dc, lse, causal=causal, scale=w.scale,
-                                                layout=layout, block_step_bwd=bs_bwd, add_and_clear=add_clear)
+                                                layout=layout, bidirectional=bi, block_step_bwd=bs_bwd,
+                                                add_and_clear=add_clear)
                 ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
                 ro = shard(torch.from_numpy(ro), rank, world, layout).numpy()
                 rl = shard(torch.from_numpy(rl), rank, world, layout, dim=2).numpy()
@@ -102,7 +105,7 @@ def _worker(rank, world, port, results):
                               for g, r_ in zip((dq, dk, dv),
                                                (shard(torch.from_numpy(x), rank, world, layout).numpy()
                                                 for x in grads)))
-                results[(rank, ci, layout)] = (float(np.max(np.abs(out.float().numpy() - ro))),
+                results[(rank, ci, layout, bi)] = (float(np.max(np.abs(out.float().numpy() - ro))),
                                                float(np.max(np.abs(lse.numpy() - rl))), g_ratio)
         torch.cuda.synchronize(dev)
     finally:
@@ -121,6 +124,6 @@ def test_ring_ranks_with_cuda_kernels_match_oracle(world):
         p.join(timeout=600)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
     got = dict(results)
-    assert sorted(got) == sorted((r, ci, lay) for r in range(world) for ci in range(len(CASES)) for lay in LAYOUTS)
+    assert sorted(got) == sorted((r, ci, lay, bi) for r in range(world) for ci in range(len(CASES)) for lay, bi in MODES)
     for key, (eo, el, gr) in got.items():
         assert eo <= 2e-2 and el <= 1e-3 and gr <= 1.0, (key, eo, el, gr)

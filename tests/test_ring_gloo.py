@@ -1,7 +1,8 @@
 """The sequence-parallel ring protocol across ranks, on CPU (gloo).
 
 Each rank holds one chunk of Q, K, V; ring_attention passes KV chunks around
-the ring and folds them into the running state.  For the CPU test the
+the ring (one-way, or both ways in the bidirectional ring) and folds them into
+the running state.  For the CPU test the
 per-visit compute is the oracle's block step (float64), so what is checked
 here is the protocol: visit order, message routing, buffer swaps, causal
 skipping and the final normalisation.  The result on every rank must equal
@@ -46,7 +47,8 @@ def _oracle_compute():
 
 
 CASES = [(1, 2, 2, 16, 8, True), (2, 4, 2, 12, 8, False), (1, 4, 1, 10, 4, True)]
-LAYOUTS = ["contiguous", "zigzag"]
+# (chunk layout, bidirectional)
+MODES = [("contiguous", False), ("zigzag", False), ("contiguous", True), ("zigzag", True)]
 
 
 def _setup(rank, world, port):
@@ -68,7 +70,7 @@ def _worker(rank, world, port, results):
         # Every case and layout in one process group (every rank takes the
         # same steps in the same order).
         for ci, case in enumerate(CASES):
-            for layout in LAYOUTS:
+            for layout, bi in MODES:
                 B, Hq, Hkv, L, d, causal = case
                 w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
                                     seed=11 + world + ci)
@@ -76,15 +78,15 @@ def _worker(rank, world, port, results):
                 bs, fin, init = _oracle_compute()
                 qc, kc, vc = (shard(x, rank, world, layout) for x in (q, k, v))
                 before = [x.clone() for x in (qc, kc, vc)]
-                out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, layout=layout, block_step=bs,
-                                          finalize=fin, init_state=init)
+                out, lse = ring_attention(qc, kc, vc, causal=causal, scale=w.scale, layout=layout, bidirectional=bi,
+                                          block_step=bs, finalize=fin, init_state=init)
                 # The ring only reads the caller's chunks.
                 assert all(torch.equal(a, b) for a, b in zip(before, (qc, kc, vc)))
                 ro, rl = oracle.attention_ref(q, k, v, causal=causal, scale=w.scale)
                 ro = shard(torch.from_numpy(ro), rank, world, layout).numpy()
                 rl = shard(torch.from_numpy(rl), rank, world, layout, dim=2).numpy()
-                results[(rank, ci, layout)] = (float(np.max(np.abs(out.numpy() - ro))),
-                                               float(np.max(np.abs(lse.numpy() - rl))))
+                results[(rank, ci, layout, bi)] = (float(np.max(np.abs(out.numpy() - ro))),
+                                                   float(np.max(np.abs(lse.numpy() - rl))))
     finally:
         dist.destroy_process_group()
 
@@ -100,7 +102,7 @@ def _run_ranks(target, world):
         p.join(timeout=300)
         assert p.exitcode == 0, f"rank exited with {p.exitcode}"
     got = dict(results)
-    assert sorted(got) == sorted((r, ci, lay) for r in range(world) for ci in range(len(CASES)) for lay in LAYOUTS)
+    assert sorted(got) == sorted((r, ci, lay, bi) for r in range(world) for ci in range(len(CASES)) for lay, bi in MODES)
     return got
 
 
@@ -136,7 +138,7 @@ def _bwd_worker(rank, world, port, results):
         from long_context_exact_blockwise_b200.ring import ring_attention_bwd, shard
 
         for ci, case in enumerate(CASES):
-            for layout in LAYOUTS:
+            for layout, bi in MODES:
                 B, Hq, Hkv, L, d, causal = case
                 w = workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=world * L, d=d, dtype="f32", causal=causal, P=world,
                                     seed=31 + world + ci)
@@ -146,11 +148,11 @@ def _bwd_worker(rank, world, port, results):
                 chunks = [shard(x, rank, world, layout) for x in (q, k, v, out, dout)]
                 before = [x.clone() for x in chunks]
                 dq, dk, dv = ring_attention_bwd(*chunks, shard(lse, rank, world, layout, dim=2), causal=causal,
-                                                scale=w.scale, layout=layout, block_step_bwd=_oracle_bwd_step(),
-                                                add_and_clear=_add_and_clear_cpu)
+                                                scale=w.scale, layout=layout, bidirectional=bi,
+                                                block_step_bwd=_oracle_bwd_step(), add_and_clear=_add_and_clear_cpu)
                 assert all(torch.equal(a, b) for a, b in zip(before, chunks))
                 rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=causal, scale=w.scale)
-                results[(rank, ci, layout)] = tuple(
+                results[(rank, ci, layout, bi)] = tuple(
                     float(np.max(np.abs(g.numpy() - shard(torch.from_numpy(r), rank, world, layout).numpy())))
                     for g, r in ((dq, rq), (dk, rk), (dv, rv)))
     finally:
@@ -161,6 +163,30 @@ def _bwd_worker(rank, world, port, results):
 def test_ring_backward_protocol_matches_full_gradient(world):
     for key, errs in _run_ranks(_bwd_worker, world).items():
         assert max(errs) <= 1e-10, (key, errs)
+
+
+def test_bidirectional_visit_order_and_pieces():
+    from long_context_exact_blockwise_b200.ring import _kv_plan, ring_visit_order_bidirectional
+    # 4 ranks: rank 1 holds the first piece of ranks 1, 2, 3, 0 (from its
+    # right-hand neighbour) and the second piece of ranks 1, 0, 3, 2 (from
+    # its left-hand neighbour).
+    assert ring_visit_order_bidirectional(1, 4) == [(1, 1), (2, 0), (3, 3), (0, 2)]
+    # Over the P steps every rank sees both pieces of every rank exactly once.
+    for world in (1, 2, 3, 5):
+        for rank in range(world):
+            order = ring_visit_order_bidirectional(rank, world)
+            assert sorted(a for a, _ in order) == list(range(world))
+            assert sorted(b for _, b in order) == list(range(world))
+    # Key offsets: contiguous halves of a 16-key chunk; zigzag chunks of 8 keys
+    # (rank 1 of 4 holds chunks 1 and 6).
+    n_k, offs = _kv_plan(1, 4, "contiguous", 16, True)
+    assert n_k == 2 and offs(0) == [16, 24] and offs(1) == [32, 8] and offs(3) == [0, 40]
+    n_k, offs = _kv_plan(1, 4, "zigzag", 16, True)
+    assert n_k == 2 and offs(0) == [8, 48] and offs(1) == [16, 56] and offs(2) == [24, 32]
+    # Every key offset appears exactly once over the ring.
+    for layout in ("contiguous", "zigzag"):
+        n_k, offs = _kv_plan(2, 4, layout, 16, True)
+        assert sorted(o for s in range(4) for o in offs(s)) == list(range(0, 64, 8))
 
 
 def test_ring_visit_order_matches_schedule_figure():
