@@ -339,17 +339,25 @@ def run_ours(args, w, rank, world, device):
             h_sc = [k_sc.cpu().pin_memory(), v_sc.cpu().pin_memory()]
             x_sc = [k_sc, v_sc]  # the call reads the scales from these device tensors
 
-        def e2e_step():
-            xq.copy_(hq, non_blocking=True)
-            xk.copy_(hk, non_blocking=True)
-            xv.copy_(hv, non_blocking=True)
-            if fp8:
-                for x, h in zip(x_sc, h_sc):
-                    x.copy_(h, non_blocking=True)
-            fn(xq, xk, xv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out,
-               lse=lse, stream=stream)
-            h_out[0].copy_(out, non_blocking=True)
-            h_out[1].copy_(lse, non_blocking=True)
+        if fn is R.ring_attn_fwd:
+            # The bf16 forward has a host-buffer entry point that streams
+            # KV-head groups through the device, copies overlapped with the
+            # compute.
+            def e2e_step():
+                R.ring_attn_fwd_host(hq, hk, hv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci,
+                                     scale=w.scale, out=h_out[0], lse=h_out[1], stream=stream)
+        else:
+            def e2e_step():
+                xq.copy_(hq, non_blocking=True)
+                xk.copy_(hk, non_blocking=True)
+                xv.copy_(hv, non_blocking=True)
+                if fp8:
+                    for x, h in zip(x_sc, h_sc):
+                        x.copy_(h, non_blocking=True)
+                fn(xq, xk, xv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out,
+                   lse=lse, stream=stream)
+                h_out[0].copy_(out, non_blocking=True)
+                h_out[1].copy_(lse, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(device)

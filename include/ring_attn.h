@@ -95,6 +95,43 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
                   void* stream);
 
 /*
+ * ring_attn_fwd_host -- ring_attn_fwd for inputs and results in HOST memory,
+ * with the copies overlapped with the compute.
+ *
+ * Attention heads are independent problems (in the definition above, every
+ * (b, h) has its own softmax over its own keys), so the call cuts the KV
+ * heads into groups of `kv_heads_per_group` (with their
+ * Hq / Hkv query heads each) and streams them through two device staging
+ * slots: while group g is computed, group g + 1 is copied in and group g - 1
+ * copied out.  A step then costs about its host-to-device transfer instead
+ * of transfer + compute + transfer back.
+ *
+ * q, k, v, out, lse: HOST pointers with the layouts of ring_attn_fwd
+ * ([B, N, H, d] bf16, lse [B, Hq, N_q] float32), owned by the caller.
+ * Page-locked memory (cudaHostAlloc / pinned tensors) is needed for the
+ * copies to overlap; pageable memory gives the same result without overlap.
+ * Other arguments as ring_attn_fwd; each group is computed exactly as
+ * ring_attn_fwd computes it (the split-KV count of an incremental query is
+ * chosen per group).
+ * kv_heads_per_group: 0 = the fewest KV heads per group that give at most
+ * sixteen groups; else it must divide Hkv (RA_ERR_INVALID_ARG otherwise).
+ *
+ * Asynchronous like ring_attn_fwd: the pipeline starts after the work queued
+ * on `stream` and `stream` waits for all of it, so out and lse are complete
+ * once `stream` has been synchronised (ring_attn_sync_status).  The caller
+ * keeps q, k, v, out and lse allocated and unmodified until then.  The library
+ * uses four internal streams per device, created on the first call, and a
+ * stream-ordered staging allocation on `stream` of
+ * 2 x (2 B N_q hg d 2 + 2 B N_kv kvg d 2 + B hg N_q 4) bytes (hg, kvg: query
+ * and KV heads per group), freed on `stream` when the pipeline ends.
+ * Returns as ring_attn_fwd; RA_ERR_OOM when the staging allocation fails.
+ */
+int ring_attn_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d,
+                       int causal, int64_t chunk, int P, int64_t cache_idx, float scale,
+                       int kv_heads_per_group, void* stream);
+
+/*
  * ring_attn_fwd_f32 -- the same operation with float32 q/k/v/out, computed
  * in float32 on CUDA cores (no TF32 tensor cores: the float32 path is held
  * to 1e-4 absolute error).  Same arguments, conventions and statuses.

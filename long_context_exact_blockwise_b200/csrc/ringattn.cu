@@ -7,6 +7,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -288,6 +289,207 @@ int ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float*
   a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0;
   a.S = cache_idx < 0 ? 1 : 0;  // 0: choose a split count
   return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd");
+}
+
+}  // extern "C"
+
+namespace {
+
+// The host-buffer pipeline's streams on one device (q in, k and v in,
+// compute, results out), created once, all or none.  Two copy-in streams let
+// the q and the k / v copies of a group run on separate copy engines.
+struct PipeStreams {
+  cudaStream_t h2d = nullptr, h2d_kv = nullptr, comp = nullptr, d2h = nullptr;
+};
+
+int pipe_streams(PipeStreams** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static PipeStreams per_dev[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  PipeStreams& p = per_dev[dev];
+  if (!p.h2d) {
+    cudaStream_t s[4] = {nullptr, nullptr, nullptr, nullptr};
+    for (int i = 0; i < 4; ++i) {
+      e = cudaStreamCreateWithFlags(&s[i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) {
+        for (int j = 0; j < i; ++j) cudaStreamDestroy(s[j]);
+        return set_cuda_error(e, "cudaStreamCreateWithFlags");
+      }
+    }
+    p.h2d = s[0];
+    p.h2d_kv = s[1];
+    p.comp = s[2];
+    p.d2h = s[3];
+  }
+  *out = &p;
+  return RA_OK;
+}
+
+// Events of one pipelined call, destroyed when the call returns (a pending
+// event's resources are released once it completes).
+struct CallEvents {
+  std::vector<cudaEvent_t> ev;
+  ~CallEvents() {
+    for (cudaEvent_t x : ev) cudaEventDestroy(x);
+  }
+  cudaError_t make(size_t n) {
+    ev.reserve(n);
+    for (size_t i = 0; i < n; ++i) {
+      cudaEvent_t x;
+      cudaError_t e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+      if (e != cudaSuccess) return e;
+      ev.push_back(x);
+    }
+    return cudaSuccess;
+  }
+};
+
+// KV heads per group when the caller passes 0: the fewest that give at most
+// sixteen groups (and divide Hkv).  On the 32-head 32K prefill, 16 groups of
+// two KV heads measured 17.7 ms per step, 8 of four 17.9, 32 of one 20.4 and
+// 4 of eight 20.0 (one copy-in stream).
+int default_kv_group(int Hkv) {
+  int g = 1;
+  while (Hkv / g > 16 || Hkv % g != 0) ++g;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ring_attn_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                       int64_t N_q, int64_t N_kv, int d, int causal, int64_t chunk, int P, int64_t cache_idx,
+                       float scale, int kv_heads_per_group, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_host");
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, chunk, P, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (kv_heads_per_group < 0 || kv_heads_per_group > Hkv ||
+      (kv_heads_per_group > 0 && Hkv % kv_heads_per_group != 0))
+    return RA_ERR_INVALID_ARG;
+  if (B == 0 || N_q == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  PipeStreams* ps = nullptr;
+  if ((r = pipe_streams(&ps)) != RA_OK) return r;
+
+  const int kvg = kv_heads_per_group > 0 ? kv_heads_per_group : default_kv_group(Hkv);
+  const int n_groups = Hkv / kvg;
+  const int hg = kvg * (Hq / Hkv);  // query heads per group
+  const int n_slots = n_groups > 1 ? 2 : 1;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t row_q = (size_t)hg * d * 2, row_kv = (size_t)kvg * d * 2;
+  const size_t q_bytes = up((size_t)B * N_q * row_q), kv_bytes = up((size_t)B * N_kv * row_kv);
+  const size_t lse_bytes = up((size_t)B * hg * N_q * 4);
+  const size_t slot_bytes = 2 * q_bytes + 2 * kv_bytes + lse_bytes;  // q, k, v, out, lse
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // Events: start, then per group (q in, k / v in, computed, copied out),
+  // then the four streams' ends.
+  CallEvents evs;
+  cudaError_t e = evs.make(1 + 4 * (size_t)n_groups + 4);
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaEventCreateWithFlags");
+  cudaEvent_t ev_start = evs.ev[0];
+  auto ev_in = [&](int g) { return evs.ev[1 + 4 * g]; };
+  auto ev_in_kv = [&](int g) { return evs.ev[2 + 4 * g]; };
+  auto ev_comp = [&](int g) { return evs.ev[3 + 4 * g]; };
+  auto ev_out = [&](int g) { return evs.ev[4 + 4 * g]; };
+  cudaEvent_t* ev_end = &evs.ev[1 + 4 * n_groups];
+
+  if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
+    t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
+    return RA_ERR_OOM;
+  }
+  void* ws = nullptr;
+  e = cudaMallocAsync(&ws, slot_bytes * n_slots, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
+    return RA_ERR_OOM;
+  }
+  // The pipeline starts after the work already queued on the caller's stream.
+  e = cudaEventRecord(ev_start, st);
+  for (cudaStream_t s : {ps->h2d, ps->h2d_kv, ps->comp, ps->d2h})
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_start, 0);
+
+  const char* qh = static_cast<const char*>(q);
+  const char* kh = static_cast<const char*>(k);
+  const char* vh = static_cast<const char*>(v);
+  char* oh = static_cast<char*>(out);
+  char* lh = reinterpret_cast<char*>(lse);
+  int status = RA_OK;
+  for (int g = 0; g < n_groups && e == cudaSuccess && status == RA_OK; ++g) {
+    char* base = static_cast<char*>(ws) + (size_t)(g % n_slots) * slot_bytes;
+    char* qd = base;
+    char* kd = qd + q_bytes;
+    char* vd = kd + kv_bytes;
+    char* od = vd + kv_bytes;
+    float* ld = reinterpret_cast<float*>(od + q_bytes);
+    // In: the group's heads of every token row, packed into the slot
+    // (once the compute of the group that used the slot before is done).
+    if (g >= n_slots) e = cudaStreamWaitEvent(ps->h2d, ev_comp(g - n_slots), 0);
+    if (e == cudaSuccess && g >= n_slots) e = cudaStreamWaitEvent(ps->h2d_kv, ev_comp(g - n_slots), 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(qd, row_q, qh + (size_t)g * row_q, (size_t)Hq * d * 2, row_q, (size_t)B * N_q,
+                            cudaMemcpyHostToDevice, ps->h2d);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(kd, row_kv, kh + (size_t)g * row_kv, (size_t)Hkv * d * 2, row_kv, (size_t)B * N_kv,
+                            cudaMemcpyHostToDevice, ps->h2d_kv);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(vd, row_kv, vh + (size_t)g * row_kv, (size_t)Hkv * d * 2, row_kv, (size_t)B * N_kv,
+                            cudaMemcpyHostToDevice, ps->h2d_kv);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in(g), ps->h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in_kv(g), ps->h2d_kv);
+    // Compute: the group is an independent problem of hg query heads over kvg
+    // KV heads (once the slot's previous results have been copied out).
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->comp, ev_in(g), 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->comp, ev_in_kv(g), 0);
+    if (e == cudaSuccess && g >= n_slots) e = cudaStreamWaitEvent(ps->comp, ev_out(g - n_slots), 0);
+    if (e != cudaSuccess) break;
+    ProblemArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = qd; a.k = kd; a.v = vd; a.out = od; a.lse = ld;
+    a.B = B; a.Hq = hg; a.Hkv = kvg; a.d = d;
+    a.N_q = N_q; a.N_kv = N_kv;
+    a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+    a.k_pos0 = 0;
+    a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0;
+    a.S = cache_idx < 0 ? 1 : 0;
+    status = run_fwd(a, num_sms, ps->comp, "ring_attn_fwd_host");
+    if (status != RA_OK) break;
+    e = cudaEventRecord(ev_comp(g), ps->comp);
+    // Out: the group's heads back into their places of every token row.
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->d2h, ev_comp(g), 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(oh + (size_t)g * row_q, (size_t)Hq * d * 2, od, row_q, row_q, (size_t)B * N_q,
+                            cudaMemcpyDeviceToHost, ps->d2h);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(lh + (size_t)g * hg * N_q * 4, (size_t)Hq * N_q * 4, ld, (size_t)hg * N_q * 4,
+                            (size_t)hg * N_q * 4, (size_t)B, cudaMemcpyDeviceToHost, ps->d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out(g), ps->d2h);
+  }
+  // Join: the caller's stream waits for all four streams (also after a
+  // failure, so the staging is freed only once nothing uses it).
+  cudaError_t ej = cudaSuccess;
+  cudaStream_t pipes[4] = {ps->h2d, ps->h2d_kv, ps->comp, ps->d2h};
+  for (int i = 0; i < 4; ++i) {
+    if (ej == cudaSuccess) ej = cudaEventRecord(ev_end[i], pipes[i]);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, ev_end[i], 0);
+  }
+  if (ej != cudaSuccess) {
+    // The join could not be queued: wait for the pipeline on the host.
+    for (cudaStream_t s : pipes) cudaStreamSynchronize(s);
+  }
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (status != RA_OK) return status;
+  if (e == cudaSuccess) e = ej;
+  if (e == cudaSuccess) e = ef;
+  return finish(e, st, "ring_attn_fwd_host");
 }
 
 int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,

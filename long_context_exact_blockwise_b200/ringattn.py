@@ -54,6 +54,7 @@ _SIGS = {
     "ring_attn_fwd": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
+    "ring_attn_fwd_host": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _i, _p],
     "ring_attn_fwd_window_anchor": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _i, _l, _i, _l, _l, _f, _p],
     "ring_attn_fwd_fp8kv": [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
@@ -174,6 +175,48 @@ def ring_attn_fwd(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None,
     """bf16 forward: q [B,N_q,Hq,d], k/v [B,N_kv,Hkv,d] -> (out bf16, lse f32 [B,Hq,N_q])."""
     return _fwd(lib.ring_attn_fwd, torch.bfloat16, q, k, v, causal, P, chunk, cache_idx, scale, out, lse,
                 stream)
+
+
+def _need_host(t: torch.Tensor, name: str, dtype: torch.dtype):
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a CPU (host) tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def ring_attn_fwd_host(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None, cache_idx=None,
+                       scale: Optional[float] = None, out=None, lse=None, kv_heads_per_group: int = 0,
+                       stream=None):
+    """bf16 forward for host tensors, copies overlapped with the compute.
+
+    q [B,N_q,Hq,d], k/v [B,N_kv,Hkv,d] are CPU tensors (pinned for overlap);
+    out / lse are CPU tensors (pinned ones are allocated if None).  The work is
+    queued on `stream` (the current CUDA stream by default): synchronise it
+    before reading out and lse.  Returns (out, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_host(t, n, torch.bfloat16)
+    B, N_q, Hq, d = q.shape
+    _, N_kv, Hkv, dk = k.shape
+    if k.shape != v.shape or dk != d or k.shape[0] != B:
+        raise ValueError("k and v must be [B, N_kv, Hkv, d] matching q")
+    if chunk is None:
+        chunk = N_kv // P if P > 0 else 0
+    ci = -1 if cache_idx is None else int(cache_idx)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, Hq, N_q), dtype=torch.float32).pin_memory()
+    _need_host(out, "out", torch.bfloat16)
+    _need_host(lse, "lse", torch.float32)
+    device = torch.cuda.current_device()
+    st = lib.ring_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N_q, N_kv, d,
+                                int(bool(causal)), int(chunk), int(P), ci, sc, int(kv_heads_per_group),
+                                _stream(stream, device))
+    _check(st, "ring_attn_fwd_host")
+    return out, lse
 
 
 def ring_attn_fwd_f32(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None, cache_idx=None,

@@ -182,3 +182,17 @@ def test_nvtx_ranges_switch_keeps_validation(monkeypatch):
     assert L.ring_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 128, 128, 96, 1, 128, 1, -1, 0.1, None) == \
         ra.RA_ERR_INVALID_ARG
     assert L.ring_attn_add_and_clear(FAKE, ctypes.c_void_p(0x20000), 0, None) == ra.RA_OK
+
+
+def test_fwd_host_validation():
+    # The host-buffer forward validates like ring_attn_fwd, and its group size
+    # must divide Hkv; all of it before any CUDA call.
+    ra = _lib()
+    L = ra.lib
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 512, 512, 128, 1, 128, 4, -1, 0.088, 0, None]
+    for i, val in ((16, -1), (16, 3), (16, 5), (10, 96), (0, None), (5, -1)):
+        bad = list(ok); bad[i] = val
+        assert L.ring_attn_fwd_host(*bad) == ra.RA_ERR_INVALID_ARG, (i, val)
+    zero_b = list(ok); zero_b[5] = 0
+    assert L.ring_attn_fwd_host(*zero_b) == ra.RA_OK  # nothing to do: no device needed
+    assert L.ring_attn_fwd_host(*ok) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
