@@ -324,12 +324,10 @@ def run_ours(args, w, rank, world, device):
         h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
 
         def e2e_step():
-            for x, h in zip(x_in, h_in):
-                x.copy_(h, non_blocking=True)
-            R.ring_attn_bwd(*x_in, causal=w.causal, cache_idx=ci, scale=w.scale, dq=dq, dk=dk, dv=dv,
-                            stream=stream)
-            for h, x in zip(h_out, (dq, dk, dv)):
-                h.copy_(x, non_blocking=True)
+            # Host-buffer backward: KV-head groups stream through the device,
+            # copies overlapped with the compute.
+            R.ring_attn_bwd_host(*h_in, causal=w.causal, cache_idx=ci, scale=w.scale, dq=h_out[0], dk=h_out[1],
+                                 dv=h_out[2], stream=stream)
     else:
         h_in = [hq, hk, hv]
         h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),

@@ -249,6 +249,28 @@ int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, voi
                                 int64_t window, int64_t anchor_period, float scale, void* stream);
 
 /*
+ * ring_attn_bwd_host -- ring_attn_bwd for inputs and results in HOST memory,
+ * with the copies overlapped with the compute, as ring_attn_fwd_host: the
+ * KV heads are cut into groups of `kv_heads_per_group` (0 = at most sixteen
+ * groups) with their query heads, and each group's q, k, v, out, dout, lse
+ * are copied in, its three backward kernels run, and its dq, dk, dv are
+ * copied out while the neighbouring groups are copied.  Each group is
+ * computed exactly as ring_attn_bwd computes those heads.
+ *
+ * Pointers: HOST memory with the layouts of ring_attn_bwd, owned by the
+ * caller, kept allocated and unmodified until `stream` has been
+ * synchronised; page-locked memory for overlap.  Staging on the device:
+ * 2 x (4 B N_q hg d 2 + 4 B N_kv kvg d 2 + B hg N_q 4) bytes plus the
+ * backward's own workspace, stream-ordered on `stream`.
+ * Returns as ring_attn_bwd; RA_ERR_INVALID_ARG also when kv_heads_per_group
+ * does not divide Hkv.
+ */
+int ring_attn_bwd_host(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
+                       int64_t cache_idx, float scale, int kv_heads_per_group, void* stream);
+
+/*
  * ring_attn_bwd_block_step -- the backward of one ring visit: adds, in
  * place, the share of dq, dk, dv that comes from the pairs of query chunk
  * q_chunk [B, Lq, Hq, d] (global positions q_off + t) and KV chunk

@@ -349,6 +349,8 @@ struct CallEvents {
   }
 };
 
+int run_bwd(ra::BwdArgs a, const char* what, cudaStream_t st);  // below
+
 // KV heads per group when the caller passes 0: the fewest that give at most
 // sixteen groups (and divide Hkv).  On the 32-head 32K prefill, 16 groups of
 // two KV heads measured 17.7 ms per step, 8 of four 17.9, 32 of one 20.4 and
@@ -357,6 +359,125 @@ int default_kv_group(int Hkv) {
   int g = 1;
   while (Hkv / g > 16 || Hkv % g != 0) ++g;
   return g;
+}
+
+// One tensor of a host-buffer pipeline.  Group g's part is `rows` rows of
+// `row_bytes` bytes starting at byte g * row_bytes of the host tensor, one
+// row every `pitch` bytes; on the device it is packed (pitch = row_bytes).
+// Inputs go in on copy-in stream `lane` (0 or 1); outputs come back after
+// the group's compute.
+struct PipeTensor {
+  const void* in;   // host input, or nullptr
+  void* out;        // host output, or nullptr
+  size_t row_bytes, pitch, rows;
+  int lane;
+};
+
+// Streams the groups of a host-buffer call through two device staging slots:
+// while group g computes, group g + 1 is copied in and group g - 1 copied out.
+// compute(g, dev, comp_stream) launches group g's work on the packed device
+// tensors dev[i] (same order as t) and returns an ra status.
+template <class F>
+int run_host_pipeline(int n_groups, const PipeTensor* t, int n_t, cudaStream_t st, const char* what, F&& compute) {
+  constexpr int kMaxTensors = 12;
+  if (n_t > kMaxTensors) return RA_ERR_INVALID_ARG;
+  PipeStreams* ps = nullptr;
+  int r = pipe_streams(&ps);
+  if (r != RA_OK) return r;
+  const int n_slots = n_groups > 1 ? 2 : 1;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  size_t off[kMaxTensors];
+  size_t slot_bytes = 0;
+  for (int i = 0; i < n_t; ++i) {
+    off[i] = slot_bytes;
+    slot_bytes += up(t[i].row_bytes * t[i].rows);
+  }
+  cudaStream_t lanes[2] = {ps->h2d, ps->h2d_kv};
+
+  // Events: start, then per group (in on each lane, computed, out), then the
+  // four streams' ends.
+  CallEvents evs;
+  cudaError_t e = evs.make(1 + 4 * (size_t)n_groups + 4);
+  if (e != cudaSuccess) return set_cuda_error(e, "cudaEventCreateWithFlags");
+  cudaEvent_t ev_start = evs.ev[0];
+  auto ev_in = [&](int g, int lane) { return evs.ev[1 + 4 * g + lane]; };
+  auto ev_comp = [&](int g) { return evs.ev[3 + 4 * g]; };
+  auto ev_out = [&](int g) { return evs.ev[4 + 4 * g]; };
+  cudaEvent_t* ev_end = &evs.ev[1 + 4 * n_groups];
+
+  if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
+    t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
+    return RA_ERR_OOM;
+  }
+  void* ws = nullptr;
+  e = cudaMallocAsync(&ws, slot_bytes * n_slots, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
+    return RA_ERR_OOM;
+  }
+  // The pipeline starts after the work already queued on the caller's stream.
+  e = cudaEventRecord(ev_start, st);
+  cudaStream_t pipes[4] = {ps->h2d, ps->h2d_kv, ps->comp, ps->d2h};
+  for (cudaStream_t s : pipes)
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_start, 0);
+
+  int status = RA_OK;
+  for (int g = 0; g < n_groups && e == cudaSuccess && status == RA_OK; ++g) {
+    char* base = static_cast<char*>(ws) + (size_t)(g % n_slots) * slot_bytes;
+    void* dev[kMaxTensors];
+    for (int i = 0; i < n_t; ++i) dev[i] = base + off[i];
+    // In, once the compute of the group that used the slot before is done.
+    for (int lane = 0; lane < 2 && e == cudaSuccess; ++lane)
+      if (g >= n_slots) e = cudaStreamWaitEvent(lanes[lane], ev_comp(g - n_slots), 0);
+    for (int i = 0; i < n_t && e == cudaSuccess; ++i)
+      if (t[i].in)
+        e = cudaMemcpy2DAsync(dev[i], t[i].row_bytes, static_cast<const char*>(t[i].in) + (size_t)g * t[i].row_bytes,
+                              t[i].pitch, t[i].row_bytes, t[i].rows, cudaMemcpyHostToDevice, lanes[t[i].lane]);
+    for (int lane = 0; lane < 2 && e == cudaSuccess; ++lane) {
+      e = cudaEventRecord(ev_in(g, lane), lanes[lane]);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->comp, ev_in(g, lane), 0);
+    }
+    // Compute, once the slot's previous results have been copied out.
+    if (e == cudaSuccess && g >= n_slots) e = cudaStreamWaitEvent(ps->comp, ev_out(g - n_slots), 0);
+    if (e != cudaSuccess) break;
+    status = compute(g, dev, ps->comp);
+    if (status != RA_OK) break;
+    e = cudaEventRecord(ev_comp(g), ps->comp);
+    // Out.
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->d2h, ev_comp(g), 0);
+    for (int i = 0; i < n_t && e == cudaSuccess; ++i)
+      if (t[i].out)
+        e = cudaMemcpy2DAsync(static_cast<char*>(t[i].out) + (size_t)g * t[i].row_bytes, t[i].pitch, dev[i],
+                              t[i].row_bytes, t[i].row_bytes, t[i].rows, cudaMemcpyDeviceToHost, ps->d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out(g), ps->d2h);
+  }
+  // Join: the caller's stream waits for all four streams (also after a
+  // failure, so the staging is freed only once nothing uses it).
+  cudaError_t ej = cudaSuccess;
+  for (int i = 0; i < 4; ++i) {
+    if (ej == cudaSuccess) ej = cudaEventRecord(ev_end[i], pipes[i]);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, ev_end[i], 0);
+  }
+  if (ej != cudaSuccess) {
+    // The join could not be queued: wait for the pipeline on the host.
+    for (cudaStream_t s : pipes) cudaStreamSynchronize(s);
+  }
+  cudaError_t ef = cudaFreeAsync(ws, st);
+  if (status != RA_OK) return status;
+  if (e == cudaSuccess) e = ej;
+  if (e == cudaSuccess) e = ef;
+  return finish(e, st, what);
+}
+
+// Host-tensor descriptors of one group: token-major [B, N, H, d] rows (the
+// group's `heads` of every token row) and [B, H, N] float32 rows (the group's
+// heads of every batch entry).
+PipeTensor token_rows(const void* in, void* out, int heads, int H, int d, size_t esz, long long BN, int lane) {
+  return PipeTensor{in, out, (size_t)heads * d * esz, (size_t)H * d * esz, (size_t)BN, lane};
+}
+PipeTensor head_rows(const void* in, void* out, int heads, int H, long long N, int B, int lane) {
+  return PipeTensor{in, out, (size_t)heads * N * 4, (size_t)H * N * 4, (size_t)B, lane};
 }
 
 }  // namespace
@@ -375,121 +496,70 @@ int ring_attn_fwd_host(const void* q, const void* k, const void* v, void* out, f
   if (B == 0 || N_q == 0) return RA_OK;
   int num_sms = 148;
   if ((r = check_device(&num_sms)) != RA_OK) return r;
-  PipeStreams* ps = nullptr;
-  if ((r = pipe_streams(&ps)) != RA_OK) return r;
-
   const int kvg = kv_heads_per_group > 0 ? kv_heads_per_group : default_kv_group(Hkv);
-  const int n_groups = Hkv / kvg;
   const int hg = kvg * (Hq / Hkv);  // query heads per group
-  const int n_slots = n_groups > 1 ? 2 : 1;
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t row_q = (size_t)hg * d * 2, row_kv = (size_t)kvg * d * 2;
-  const size_t q_bytes = up((size_t)B * N_q * row_q), kv_bytes = up((size_t)B * N_kv * row_kv);
-  const size_t lse_bytes = up((size_t)B * hg * N_q * 4);
-  const size_t slot_bytes = 2 * q_bytes + 2 * kv_bytes + lse_bytes;  // q, k, v, out, lse
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  // Events: start, then per group (q in, k / v in, computed, copied out),
-  // then the four streams' ends.
-  CallEvents evs;
-  cudaError_t e = evs.make(1 + 4 * (size_t)n_groups + 4);
-  if (e != cudaSuccess) return set_cuda_error(e, "cudaEventCreateWithFlags");
-  cudaEvent_t ev_start = evs.ev[0];
-  auto ev_in = [&](int g) { return evs.ev[1 + 4 * g]; };
-  auto ev_in_kv = [&](int g) { return evs.ev[2 + 4 * g]; };
-  auto ev_comp = [&](int g) { return evs.ev[3 + 4 * g]; };
-  auto ev_out = [&](int g) { return evs.ev[4 + 4 * g]; };
-  cudaEvent_t* ev_end = &evs.ev[1 + 4 * n_groups];
-
-  if (std::strcmp(env_str("RINGATTN_FAULT"), "alloc") == 0) {
-    t_last_error = "workspace allocation refused (RINGATTN_FAULT=alloc)";
-    return RA_ERR_OOM;
-  }
-  void* ws = nullptr;
-  e = cudaMallocAsync(&ws, slot_bytes * n_slots, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    t_last_error = std::string("cudaMallocAsync: ") + cudaGetErrorString(e);
-    return RA_ERR_OOM;
-  }
-  // The pipeline starts after the work already queued on the caller's stream.
-  e = cudaEventRecord(ev_start, st);
-  for (cudaStream_t s : {ps->h2d, ps->h2d_kv, ps->comp, ps->d2h})
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_start, 0);
-
-  const char* qh = static_cast<const char*>(q);
-  const char* kh = static_cast<const char*>(k);
-  const char* vh = static_cast<const char*>(v);
-  char* oh = static_cast<char*>(out);
-  char* lh = reinterpret_cast<char*>(lse);
-  int status = RA_OK;
-  for (int g = 0; g < n_groups && e == cudaSuccess && status == RA_OK; ++g) {
-    char* base = static_cast<char*>(ws) + (size_t)(g % n_slots) * slot_bytes;
-    char* qd = base;
-    char* kd = qd + q_bytes;
-    char* vd = kd + kv_bytes;
-    char* od = vd + kv_bytes;
-    float* ld = reinterpret_cast<float*>(od + q_bytes);
-    // In: the group's heads of every token row, packed into the slot
-    // (once the compute of the group that used the slot before is done).
-    if (g >= n_slots) e = cudaStreamWaitEvent(ps->h2d, ev_comp(g - n_slots), 0);
-    if (e == cudaSuccess && g >= n_slots) e = cudaStreamWaitEvent(ps->h2d_kv, ev_comp(g - n_slots), 0);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(qd, row_q, qh + (size_t)g * row_q, (size_t)Hq * d * 2, row_q, (size_t)B * N_q,
-                            cudaMemcpyHostToDevice, ps->h2d);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(kd, row_kv, kh + (size_t)g * row_kv, (size_t)Hkv * d * 2, row_kv, (size_t)B * N_kv,
-                            cudaMemcpyHostToDevice, ps->h2d_kv);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(vd, row_kv, vh + (size_t)g * row_kv, (size_t)Hkv * d * 2, row_kv, (size_t)B * N_kv,
-                            cudaMemcpyHostToDevice, ps->h2d_kv);
-    if (e == cudaSuccess) e = cudaEventRecord(ev_in(g), ps->h2d);
-    if (e == cudaSuccess) e = cudaEventRecord(ev_in_kv(g), ps->h2d_kv);
-    // Compute: the group is an independent problem of hg query heads over kvg
-    // KV heads (once the slot's previous results have been copied out).
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->comp, ev_in(g), 0);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->comp, ev_in_kv(g), 0);
-    if (e == cudaSuccess && g >= n_slots) e = cudaStreamWaitEvent(ps->comp, ev_out(g - n_slots), 0);
-    if (e != cudaSuccess) break;
+  const PipeTensor t[5] = {
+      token_rows(q, nullptr, hg, Hq, d, 2, (long long)B * N_q, 0),
+      token_rows(k, nullptr, kvg, Hkv, d, 2, (long long)B * N_kv, 1),
+      token_rows(v, nullptr, kvg, Hkv, d, 2, (long long)B * N_kv, 1),
+      token_rows(nullptr, out, hg, Hq, d, 2, (long long)B * N_q, 0),
+      head_rows(nullptr, lse, hg, Hq, N_q, B, 0),
+  };
+  auto compute = [&](int, void** dev, cudaStream_t cs) {
+    // The group is an independent problem of hg query heads over kvg KV heads.
     ProblemArgs a;
     std::memset(&a, 0, sizeof(a));
-    a.q = qd; a.k = kd; a.v = vd; a.out = od; a.lse = ld;
+    a.q = dev[0]; a.k = dev[1]; a.v = dev[2]; a.out = dev[3]; a.lse = static_cast<float*>(dev[4]);
     a.B = B; a.Hq = hg; a.Hkv = kvg; a.d = d;
     a.N_q = N_q; a.N_kv = N_kv;
     a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
     a.k_pos0 = 0;
     a.causal = causal; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0;
     a.S = cache_idx < 0 ? 1 : 0;
-    status = run_fwd(a, num_sms, ps->comp, "ring_attn_fwd_host");
-    if (status != RA_OK) break;
-    e = cudaEventRecord(ev_comp(g), ps->comp);
-    // Out: the group's heads back into their places of every token row.
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ps->d2h, ev_comp(g), 0);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(oh + (size_t)g * row_q, (size_t)Hq * d * 2, od, row_q, row_q, (size_t)B * N_q,
-                            cudaMemcpyDeviceToHost, ps->d2h);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(lh + (size_t)g * hg * N_q * 4, (size_t)Hq * N_q * 4, ld, (size_t)hg * N_q * 4,
-                            (size_t)hg * N_q * 4, (size_t)B, cudaMemcpyDeviceToHost, ps->d2h);
-    if (e == cudaSuccess) e = cudaEventRecord(ev_out(g), ps->d2h);
-  }
-  // Join: the caller's stream waits for all four streams (also after a
-  // failure, so the staging is freed only once nothing uses it).
-  cudaError_t ej = cudaSuccess;
-  cudaStream_t pipes[4] = {ps->h2d, ps->h2d_kv, ps->comp, ps->d2h};
-  for (int i = 0; i < 4; ++i) {
-    if (ej == cudaSuccess) ej = cudaEventRecord(ev_end[i], pipes[i]);
-    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, ev_end[i], 0);
-  }
-  if (ej != cudaSuccess) {
-    // The join could not be queued: wait for the pipeline on the host.
-    for (cudaStream_t s : pipes) cudaStreamSynchronize(s);
-  }
-  cudaError_t ef = cudaFreeAsync(ws, st);
-  if (status != RA_OK) return status;
-  if (e == cudaSuccess) e = ej;
-  if (e == cudaSuccess) e = ef;
-  return finish(e, st, "ring_attn_fwd_host");
+    return run_fwd(a, num_sms, cs, "ring_attn_fwd_host");
+  };
+  return run_host_pipeline(Hkv / kvg, t, 5, static_cast<cudaStream_t>(stream), "ring_attn_fwd_host", compute);
+}
+
+int ring_attn_bwd_host(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t N_q,
+                       int64_t N_kv, int d, int causal, int64_t cache_idx, float scale, int kv_heads_per_group,
+                       void* stream) {
+  NvtxScope nvtx_scope("ring_attn_bwd_host");
+  if (!dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
+  if (!(aligned16(dout) && aligned16(dq) && aligned16(dk) && aligned16(dv))) return RA_ERR_INVALID_ARG;
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N_q, N_kv, d, causal, N_kv, 1, cache_idx, scale, true);
+  if (r != RA_OK) return r;
+  if (kv_heads_per_group < 0 || kv_heads_per_group > Hkv ||
+      (kv_heads_per_group > 0 && Hkv % kv_heads_per_group != 0))
+    return RA_ERR_INVALID_ARG;
+  if (B == 0 || N_q == 0) return RA_OK;
+  if ((r = check_device(nullptr)) != RA_OK) return r;
+  const int kvg = kv_heads_per_group > 0 ? kv_heads_per_group : default_kv_group(Hkv);
+  const int hg = kvg * (Hq / Hkv);
+  const long long BNq = (long long)B * N_q, BNk = (long long)B * N_kv;
+  const PipeTensor t[9] = {
+      token_rows(q, nullptr, hg, Hq, d, 2, BNq, 0),      token_rows(k, nullptr, kvg, Hkv, d, 2, BNk, 1),
+      token_rows(v, nullptr, kvg, Hkv, d, 2, BNk, 1),    token_rows(out, nullptr, hg, Hq, d, 2, BNq, 0),
+      token_rows(dout, nullptr, hg, Hq, d, 2, BNq, 1),   head_rows(lse, nullptr, hg, Hq, N_q, B, 0),
+      token_rows(nullptr, dq, hg, Hq, d, 2, BNq, 0),     token_rows(nullptr, dk, kvg, Hkv, d, 2, BNk, 0),
+      token_rows(nullptr, dv, kvg, Hkv, d, 2, BNk, 0),
+  };
+  auto compute = [&](int, void** dev, cudaStream_t cs) {
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = dev[0]; a.k = dev[1]; a.v = dev[2]; a.out = dev[3]; a.dout = dev[4];
+    a.lse = static_cast<const float*>(dev[5]);
+    a.dq = dev[6]; a.dk = dev[7]; a.dv = dev[8];
+    a.B = B; a.Hq = hg; a.Hkv = kvg; a.d = d;
+    a.N_q = N_q; a.N_kv = N_kv;
+    a.q_pos0 = cache_idx < 0 ? 0 : cache_idx;
+    a.k_pos0 = 0;
+    a.causal = causal; a.scale = scale;
+    a.accumulate = 0;
+    return run_bwd(a, "ring_attn_bwd_host", cs);
+  };
+  return run_host_pipeline(Hkv / kvg, t, 9, static_cast<cudaStream_t>(stream), "ring_attn_bwd_host", compute);
 }
 
 int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,

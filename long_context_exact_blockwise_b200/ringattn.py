@@ -55,6 +55,7 @@ _SIGS = {
     "ring_attn_fwd_f32": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_noalloc": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_fwd_host": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _i, _p],
+    "ring_attn_bwd_host": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _i, _p],
     "ring_attn_fwd_window_anchor": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _i, _l, _i, _l, _l, _f, _p],
     "ring_attn_fwd_fp8kv": [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
@@ -217,6 +218,31 @@ def ring_attn_fwd_host(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = 
                                 _stream(stream, device))
     _check(st, "ring_attn_fwd_host")
     return out, lse
+
+
+def ring_attn_bwd_host(q, k, v, out, dout, lse, *, causal: bool, cache_idx=None, scale: Optional[float] = None,
+                       dq=None, dk=None, dv=None, kv_heads_per_group: int = 0, stream=None):
+    """Gradients of ring_attn_fwd's output for host tensors, copies overlapped
+    with the compute.  Inputs are CPU tensors (pinned for overlap); dq / dk /
+    dv are CPU tensors (pinned ones are allocated if None).  Synchronise
+    `stream` before reading them.  Returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need_host(t, n, torch.bfloat16)
+    _need_host(lse, "lse", torch.float32)
+    B, N_q, Hq, d = q.shape
+    _, N_kv, Hkv, _ = k.shape
+    dq = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() if dq is None else dq
+    dk = torch.empty(k.shape, dtype=torch.bfloat16).pin_memory() if dk is None else dk
+    dv = torch.empty(v.shape, dtype=torch.bfloat16).pin_memory() if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need_host(t, n, torch.bfloat16)
+    ci = -1 if cache_idx is None else int(cache_idx)
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.ring_attn_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, Hq, Hkv, N_q, N_kv, d, int(bool(causal)), ci, sc,
+                                int(kv_heads_per_group), _stream(stream, torch.cuda.current_device()))
+    _check(st, "ring_attn_bwd_host")
+    return dq, dk, dv
 
 
 def ring_attn_fwd_f32(q, k, v, *, causal: bool, P: int, chunk: Optional[int] = None, cache_idx=None,

@@ -1,4 +1,5 @@
-"""GPU parity of the host-buffer forward (ring_attn_fwd_host).
+"""GPU parity of the host-buffer forward and backward (ring_attn_fwd_host,
+ring_attn_bwd_host).
 
 Inputs and results live in host memory; the library streams KV-head groups
 through device staging slots with the copies overlapped with the compute.
@@ -125,3 +126,49 @@ def test_host_rejects_device_tensors_and_bad_groups():
     hq, hk, hv = (_host(x) for x in (q, k, v))
     with pytest.raises(R.RingAttnError):
         R.ring_attn_fwd_host(hq, hk, hv, causal=True, P=1, kv_heads_per_group=3)
+
+
+BWD = [
+    # (B, Hq, Hkv, N_q, N_kv, cache_idx, d, causal, kv heads per group)
+    (1, 8, 8, 640, 640, -1, 128, True, 0),     # default: 8 groups
+    (1, 8, 2, 384, 384, -1, 64, False, 1),     # GQA 4, two groups
+    (2, 4, 4, 200, 200, -1, 128, True, 2),     # ragged, B = 2
+]
+
+
+def _bwd_inputs(w):
+    R = ra()
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    ci = None if w.cache_idx < 0 else w.cache_idx
+    out, lse = R.ring_attn_fwd(q, k, v, causal=w.causal, P=1, cache_idx=ci, scale=w.scale)
+    g = torch.Generator(device="cuda").manual_seed(w.N_q + 17)
+    dout = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    return q, k, v, out, dout, lse
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N_q,N_kv,ci,d,causal,kvg", BWD)
+def test_host_backward_is_bit_identical_to_device(B, Hq, Hkv, N_q, N_kv, ci, d, causal, kvg):
+    R = ra()
+    w = W(B=B, Hq=Hq, Hkv=Hkv, N_q=N_q, N_kv=N_kv, cache_idx=ci, d=d, causal=causal, P=1, seed=990 + N_q + kvg)
+    xs = _bwd_inputs(w)
+    cci = None if ci < 0 else ci
+    dq, dk, dv = R.ring_attn_bwd(*xs, causal=causal, cache_idx=cci, scale=w.scale)
+    hs = [_host(x) for x in xs]
+    hq, hk, hv = R.ring_attn_bwd_host(*hs, causal=causal, cache_idx=cci, scale=w.scale, kv_heads_per_group=kvg)
+    assert R.ring_attn_sync_status() == 0
+    for got, ref in ((hq, dq), (hk, dk), (hv, dv)):
+        assert torch.equal(got.view(torch.int16), ref.cpu().view(torch.int16))
+
+
+def test_host_backward_incremental_matches_oracle():
+    R = ra()
+    w = W(B=1, Hq=4, Hkv=2, N_q=96, N_kv=512, cache_idx=416, d=128, causal=True, P=1, seed=997)
+    xs = _bwd_inputs(w)
+    hs = [_host(x) for x in xs]
+    dq, dk, dv = R.ring_attn_bwd_host(*hs, causal=True, cache_idx=416, scale=w.scale, kv_heads_per_group=1)
+    assert R.ring_attn_sync_status() == 0
+    q, k, v, out, dout, lse = xs
+    rq, rk, rv = oracle.attention_bwd_ref(q, k, v, dout, causal=True, scale=w.scale, cache_idx=416)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        err = np.abs(got.float().numpy() - ref) / (2e-2 + 2e-2 * np.abs(ref))
+        assert float(err.max()) <= 1.0
