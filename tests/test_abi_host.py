@@ -196,3 +196,15 @@ def test_fwd_host_validation():
     zero_b = list(ok); zero_b[5] = 0
     assert L.ring_attn_fwd_host(*zero_b) == ra.RA_OK  # nothing to do: no device needed
     assert L.ring_attn_fwd_host(*ok) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
+
+
+def test_bwd_host_validation():
+    ra = _lib()
+    L = ra.lib
+    ok = [FAKE] * 9 + [1, 8, 4, 512, 512, 128, 1, -1, 0.088, 0, None]
+    for i, val in ((18, -1), (18, 3), (18, 8), (14, 96), (4, None), (8, None), (6, ctypes.c_void_p(0x10008))):
+        bad = list(ok); bad[i] = val
+        assert L.ring_attn_bwd_host(*bad) == ra.RA_ERR_INVALID_ARG, (i, val)
+    zero_b = list(ok); zero_b[9] = 0
+    assert L.ring_attn_bwd_host(*zero_b) == ra.RA_OK
+    assert L.ring_attn_bwd_host(*ok) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
