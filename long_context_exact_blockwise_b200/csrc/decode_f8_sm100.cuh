@@ -81,6 +81,25 @@ __device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint32_t& hi, u
   lo = e4m3x2_rn((x0 - h.x) * 16.f, (x1 - h.y) * 16.f);
 }
 
+// Maximum of x over the 32 lanes of the warp (one reduction instruction).
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float m;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(x));
+  return m;
+}
+
+// 4 x 4 byte transpose among the four lanes of a lane quad: lane i of the quad
+// holds byte r of word x for (its key, row r); on return it holds byte k for
+// (key k of the quad, row i).  Two exchanges, each followed by a byte select.
+__device__ __forceinline__ uint32_t quad_byte_transpose(uint32_t x, int lane) {
+  const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;  // odd: y1 x1 y3 x3; even: x0 y0 x2 y2
+  const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;  // upper pair: y2 y3 x2 x3; lower: x0 x1 y0 y1
+  uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, 1);
+  x = __byte_perm(x, y, sel1);
+  y = __shfl_xor_sync(0xFFFFFFFFu, x, 2);
+  return __byte_perm(x, y, sel2);
+}
+
 // Instruction descriptor, kind::f8f6f4 with E4M3 A and B and an f32
 // accumulator (A / B formats 0 = E4M3); a_mn / b_mn: operand is MN-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, int b_mn) {
@@ -386,9 +405,7 @@ __global__ void __launch_bounds__(384, MINB) decode_f8_sm100_kernel(const __grid
         }
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          float m = xv[c];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          const float m = warp_max_f32(xv[c]);
           if (lane == 0) rb[(c0 + c) * 4 + quad] = m;
         }
       }
@@ -444,11 +461,11 @@ __global__ void __launch_bounds__(384, MINB) decode_f8_sm100_kernel(const __grid
         }
       }
       // P planes of buffer bsel (last read by PV_{j-2}): K-major, 128-byte
-      // swizzle; row n, key `row` at n * 128 + ((row / 16) ^ (n mod 8)) * 16 +
-      // row mod 16.
-      if (j >= 2 && !(ok = mbar_wait_idle(BAR_PV(bsel), ((j - 2) >> 1) & 1u, abort_flag))) break;
-      uint8_t* pbuf = smem + L::kPOff + bsel * L::kPBytes;
-      const int kc = row >> 4, kb = row & 15;
+      // swizzle; row n, key k at n * 128 + ((k / 16) ^ (n mod 8)) * 16 +
+      // k mod 16.  A thread's codes for 4 consecutive rows form one word; a
+      // byte transpose in each lane quad turns them into 4 consecutive keys
+      // of one row, stored as one 32-bit word.
+      uint32_t whi[CH / 4], wlo[CH / 4];
 #pragma unroll
       for (int c = 0; c < CH; c += 2) {
         const float p0 = ex2(xv[c] - (m2[c] == -INFINITY ? 0.f : m2[c]));
@@ -457,11 +474,23 @@ __global__ void __launch_bounds__(384, MINB) decode_f8_sm100_kernel(const __grid
         lsum[c + 1] += p1;
         uint32_t hi, lo;
         split_e4m3x2(p0, p1, hi, lo);
-        const int r0 = c0 + c, r1 = c0 + c + 1, s0 = NR + c0 + c, s1 = NR + c0 + c + 1;
-        pbuf[r0 * 128 + ((kc ^ (r0 & 7)) << 4) + kb] = (uint8_t)(hi & 0xFFu);
-        pbuf[r1 * 128 + ((kc ^ (r1 & 7)) << 4) + kb] = (uint8_t)(hi >> 8);
-        pbuf[s0 * 128 + ((kc ^ (s0 & 7)) << 4) + kb] = (uint8_t)(lo & 0xFFu);
-        pbuf[s1 * 128 + ((kc ^ (s1 & 7)) << 4) + kb] = (uint8_t)(lo >> 8);
+        if ((c & 2) == 0) {
+          whi[c / 4] = hi;
+          wlo[c / 4] = lo;
+        } else {
+          whi[c / 4] |= hi << 16;
+          wlo[c / 4] |= lo << 16;
+        }
+      }
+      if (j >= 2 && !(ok = mbar_wait_idle(BAR_PV(bsel), ((j - 2) >> 1) & 1u, abort_flag))) break;
+      uint8_t* pbuf = smem + L::kPOff + bsel * L::kPBytes;
+      const int k4 = quad * 32 + 4 * (lane >> 2);  // first of the quad's 4 keys
+#pragma unroll
+      for (int h = 0; h < CH / 4; ++h) {
+        const int nh = c0 + 4 * h + (lane & 3), nl = NR + nh;
+        const uint32_t th = quad_byte_transpose(whi[h], lane), tl = quad_byte_transpose(wlo[h], lane);
+        *reinterpret_cast<uint32_t*>(pbuf + nh * 128 + (((k4 >> 4) ^ (nh & 7)) << 4) + (k4 & 15)) = th;
+        *reinterpret_cast<uint32_t*>(pbuf + nl * 128 + (((k4 >> 4) ^ (nl & 7)) << 4) + (k4 & 15)) = tl;
       }
       fence_proxy_async_smem();
       tc_fence_before();

@@ -22,11 +22,24 @@ def ra():
     return m
 
 
-def run_fwd(w: workloads.Workload, device="cuda"):
-    """Run the library's forward on workload w; returns (q, k, v, out, lse) on device."""
+def run_fwd(w: workloads.Workload, device="cuda", host=False):
+    """Run the library's forward on workload w; returns (q, k, v, out, lse).
+    host=True goes through ring_attn_fwd_host (pinned host buffers, default
+    groups, as the benchmark's end-to-end line); out and lse are then on the
+    host."""
     q, k, v = workloads.make_qkv(w, device=device)
     R = ra()
     ci = None if w.cache_idx < 0 else w.cache_idx
+    if host:
+        assert w.dtype == "bf16"
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        out = torch.full(q.shape, float("nan"), dtype=q.dtype).pin_memory()
+        lse = torch.full((w.B, w.Hq, w.N_q), float("nan"), dtype=torch.float32).pin_memory()
+        R.ring_attn_fwd_host(hq, hk, hv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci, scale=w.scale, out=out,
+                             lse=lse)
+        torch.cuda.synchronize()
+        assert R.ring_attn_sync_status() == 0, "device status word set"
+        return q, k, v, out, lse
     out = torch.full_like(q, float("nan"))
     lse = torch.full((w.B, w.Hq, w.N_q), float("nan"), device=device, dtype=torch.float32)
     fn = R.ring_attn_fwd_f32 if w.dtype == "f32" else R.ring_attn_fwd
@@ -51,9 +64,10 @@ def compare(got_out, got_lse, ref_out, ref_lse, dtype: str, what: str):
     return e_out, e_lse
 
 
-def check_workload(w: workloads.Workload, rows=None, heads=None):
-    """Full-tensor parity when rows/heads are None, else on the sampled rows/heads."""
-    q, k, v, out, lse = run_fwd(w)
+def check_workload(w: workloads.Workload, rows=None, heads=None, host=False):
+    """Full-tensor parity when rows/heads are None, else on the sampled rows/heads
+    (host=True: through the host-buffer forward)."""
+    q, k, v, out, lse = run_fwd(w, host=host)
     if rows is None and heads is None:
         ro, rl = oracle.attention_ref(q, k, v, causal=w.causal, scale=w.scale, cache_idx=w.cache_idx)
         return compare(out, lse, ro, rl, w.dtype, w.name)

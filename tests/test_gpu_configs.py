@@ -42,3 +42,16 @@ def test_config5_cache_idx_sampled():
 def test_config5_decode_shapes(key):
     w = workloads.CONFIGS[key]
     check_workload(w, rows=np.arange(w.N_q), heads=[0, 1, 2, 3, 17, 31])
+
+
+# The benchmark's end-to-end line runs the bf16 forward through the
+# host-buffer entry point (KV-head groups streamed through the device).
+def test_config2_host_path_sampled():
+    w = workloads.CONFIGS[2]
+    check_workload(w, rows=sample_rows(w, n_random=64), heads=[0, 2, 3, 17, 30, 31], host=True)
+
+
+def test_config5_host_path_sampled():
+    w = workloads.CONFIGS[5]
+    rows = np.array(list(range(0, 24)) + list(range(500, 512)), dtype=np.int64)
+    check_workload(w, rows=rows, heads=[0, 3, 4, 31], host=True)
