@@ -53,19 +53,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.828320 GB read + 0.253901 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.082221056e9, "src": "4e9287c179a0d8d2"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073936 GB read + 0.004240 GB written.
-    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.078175488e9, "src": "fa8b792e8808ecd6"},
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.830061 GB read + 0.253966 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.08402688e9, "src": "bec148d66a3c98b0"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073925 GB read + 0.004619 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.07854464e9, "src": "ffc6d1b8e6968136"},
     # The full-length decodes scale the quarter-length captures by their 4x KV
     # length (traffic is K/V streaming, proportional to N_kv).
-    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.078175488e9, "src": "fa8b792e8808ecd6"},
-    # profiles/decode_f8_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537039 GB read + 0.004585 GB written.
-    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.541623808e9, "src": "fa8b792e8808ecd6"},
-    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.541623808e9, "src": "fa8b792e8808ecd6"},
-    # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step (prep + dK/dV + dQ):
-    # 0.541 + 0.011, 1.085 + 0.505, 1.084 + 0.252 GB read + written.
-    "llama7b_prefill_N32768 bwd": {"bytes": 3.477207552e9, "src": "ae663e30030606ff"},
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.07854464e9, "src": "ffc6d1b8e6968136"},
+    # profiles/decode_f8_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537022 GB read + 0.003748 GB written.
+    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.540770304e9, "src": "ffc6d1b8e6968136"},
+    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.540770304e9, "src": "ffc6d1b8e6968136"},
+    # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step, one capture
+    # per kernel (prep, dK/dV, dQ): 0.541 + 0.011, 1.084 + 0.508, 1.084 + 0.255 GB
+    # read + written.
+    "llama7b_prefill_N32768 bwd": {"bytes": 3.48383488e9, "src": "34dfa46d381e0880"},
 }
 
 
