@@ -345,6 +345,11 @@ def run_ours(args, w, rank, world, device):
             def e2e_step():
                 R.ring_attn_fwd_host(hq, hk, hv, causal=w.causal, P=w.P, chunk=w.chunk, cache_idx=ci,
                                      scale=w.scale, out=h_out[0], lse=h_out[1], stream=stream)
+        elif w.window >= 0:
+            def e2e_step():
+                R.ring_attn_fwd_window_anchor_host(hq, hk, hv, window=w.window, anchor_period=w.anchor_period,
+                                                   P=w.P, chunk=w.chunk, scale=w.scale, out=h_out[0], lse=h_out[1],
+                                                   stream=stream)
         else:
             def e2e_step():
                 xq.copy_(hq, non_blocking=True)

@@ -249,6 +249,20 @@ int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, voi
                                 int64_t window, int64_t anchor_period, float scale, void* stream);
 
 /*
+ * ring_attn_fwd_window_anchor_host -- ring_attn_fwd_window_anchor for inputs
+ * and results in HOST memory, with the copies overlapped with the compute
+ * exactly as ring_attn_fwd_host (KV-head groups of `kv_heads_per_group`,
+ * 0 = at most sixteen groups, streamed through two device staging slots).
+ * The mask is per (query, key) position, so each group is computed exactly as
+ * ring_attn_fwd_window_anchor computes those heads.  Pointers, lifetimes,
+ * staging and returns as ring_attn_fwd_host.
+ */
+int ring_attn_fwd_window_anchor_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                                     int B, int Hq, int Hkv, int64_t N, int d, int64_t chunk, int P,
+                                     int64_t window, int64_t anchor_period, float scale,
+                                     int kv_heads_per_group, void* stream);
+
+/*
  * ring_attn_bwd_host -- ring_attn_bwd for inputs and results in HOST memory,
  * with the copies overlapped with the compute, as ring_attn_fwd_host: the
  * KV heads are cut into groups of `kv_heads_per_group` (0 = at most sixteen

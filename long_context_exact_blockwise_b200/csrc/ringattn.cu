@@ -586,6 +586,45 @@ int ring_attn_fwd_window_anchor(const void* q, const void* k, const void* v, voi
   return run_fwd(a, num_sms, static_cast<cudaStream_t>(stream), "ring_attn_fwd_window_anchor");
 }
 
+int ring_attn_fwd_window_anchor_host(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                                     int Hq, int Hkv, int64_t N, int d, int64_t chunk, int P, int64_t window,
+                                     int64_t anchor_period, float scale, int kv_heads_per_group, void* stream) {
+  NvtxScope nvtx_scope("ring_attn_fwd_window_anchor_host");
+  if (window < 0 || window > kMaxTokens || anchor_period <= 0 || anchor_period % 256 != 0 ||
+      anchor_period > kMaxTokens)
+    return RA_ERR_INVALID_ARG;
+  int r = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, N, N, d, 0, chunk, P, -1, scale, true);
+  if (r != RA_OK) return r;
+  if (kv_heads_per_group < 0 || kv_heads_per_group > Hkv ||
+      (kv_heads_per_group > 0 && Hkv % kv_heads_per_group != 0))
+    return RA_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return RA_OK;
+  int num_sms = 148;
+  if ((r = check_device(&num_sms)) != RA_OK) return r;
+  const int kvg = kv_heads_per_group > 0 ? kv_heads_per_group : default_kv_group(Hkv);
+  const int hg = kvg * (Hq / Hkv);
+  const long long BN = (long long)B * N;
+  const PipeTensor t[5] = {
+      token_rows(q, nullptr, hg, Hq, d, 2, BN, 0),  token_rows(k, nullptr, kvg, Hkv, d, 2, BN, 1),
+      token_rows(v, nullptr, kvg, Hkv, d, 2, BN, 1), token_rows(nullptr, out, hg, Hq, d, 2, BN, 0),
+      head_rows(nullptr, lse, hg, Hq, N, B, 0),
+  };
+  auto compute = [&](int, void** dev, cudaStream_t cs) {
+    ProblemArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = dev[0]; a.k = dev[1]; a.v = dev[2]; a.out = dev[3]; a.lse = static_cast<float*>(dev[4]);
+    a.B = B; a.Hq = hg; a.Hkv = kvg; a.d = d;
+    a.N_q = N; a.N_kv = N;
+    a.q_pos0 = 0; a.k_pos0 = 0;
+    a.causal = 0; a.scale = scale; a.chunk = chunk; a.P = P; a.out_f32 = 0; a.S = 1;
+    a.wa_window = (int)window;
+    a.wa_period = (int)anchor_period;
+    return run_fwd(a, num_sms, cs, "ring_attn_fwd_window_anchor_host");
+  };
+  return run_host_pipeline(Hkv / kvg, t, 5, static_cast<cudaStream_t>(stream), "ring_attn_fwd_window_anchor_host",
+                           compute);
+}
+
 int ring_attn_fwd_fp8kv(const void* q, const void* k8, const void* v8, const float* k_scale, const float* v_scale,
                         void* out, float* lse, int B, int Hq, int Hkv, int64_t N_q, int64_t N_kv, int d, int causal,
                         int64_t chunk, int P, int64_t cache_idx, float scale, void* stream) {

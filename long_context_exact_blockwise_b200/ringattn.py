@@ -57,6 +57,7 @@ _SIGS = {
     "ring_attn_fwd_host": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _i, _p],
     "ring_attn_bwd_host": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _i, _p],
     "ring_attn_fwd_window_anchor": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _i, _l, _i, _l, _l, _f, _p],
+    "ring_attn_fwd_window_anchor_host": [_p, _p, _p, _p, _p, _i, _i, _i, _l, _i, _l, _i, _l, _l, _f, _i, _p],
     "ring_attn_fwd_fp8kv": [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _i, _l, _f, _p],
     "ring_attn_bwd": [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _l, _f, _p],
     "ring_attn_bwd_block_step": [_p, _p, _p, _p, _p, _p, _l, _l, _p, _p, _p, _i, _i, _i, _l, _l, _i, _i, _f, _p],
@@ -313,6 +314,31 @@ def ring_attn_fwd_window_anchor(q, k, v, *, window: int, anchor_period: int, P: 
                                          int(chunk), int(P), int(window), int(anchor_period), sc,
                                          _stream(stream, q.device))
     _check(st, "ring_attn_fwd_window_anchor")
+    return out, lse
+
+
+def ring_attn_fwd_window_anchor_host(q, k, v, *, window: int, anchor_period: int, P: int = 1,
+                                     chunk: Optional[int] = None, scale: Optional[float] = None, out=None, lse=None,
+                                     kv_heads_per_group: int = 0, stream=None):
+    """ring_attn_fwd_window_anchor for host tensors, copies overlapped with the
+    compute (as ring_attn_fwd_host).  Synchronise `stream` before reading
+    out and lse.  Returns (out, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_host(t, n, torch.bfloat16)
+    B, N, Hq, d = q.shape
+    _, N_kv, Hkv, _ = k.shape
+    if N_kv != N or v.shape != k.shape:
+        raise ValueError("the window-and-anchor mask needs N_q == N_kv")
+    chunk = N // P if chunk is None else chunk
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory() if lse is None else lse
+    _need_host(out, "out", torch.bfloat16)
+    _need_host(lse, "lse", torch.float32)
+    st = lib.ring_attn_fwd_window_anchor_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                                              int(chunk), int(P), int(window), int(anchor_period), sc,
+                                              int(kv_heads_per_group), _stream(stream, torch.cuda.current_device()))
+    _check(st, "ring_attn_fwd_window_anchor_host")
     return out, lse
 
 

@@ -208,3 +208,13 @@ def test_bwd_host_validation():
     zero_b = list(ok); zero_b[9] = 0
     assert L.ring_attn_bwd_host(*zero_b) == ra.RA_OK
     assert L.ring_attn_bwd_host(*ok) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here
+
+
+def test_window_anchor_host_validation():
+    ra = _lib()
+    L = ra.lib
+    ok = [FAKE] * 5 + [1, 8, 4, 1024, 128, 256, 4, 300, 256, 0.088, 0, None]
+    for i, val in ((15, -1), (15, 3), (13, 100), (12, -1), (9, 96), (0, None)):
+        bad = list(ok); bad[i] = val
+        assert L.ring_attn_fwd_window_anchor_host(*bad) == ra.RA_ERR_INVALID_ARG, (i, val)
+    assert L.ring_attn_fwd_window_anchor_host(*ok) == ra.RA_ERR_UNSUPPORTED  # valid, but no GPU here

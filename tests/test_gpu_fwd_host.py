@@ -172,3 +172,29 @@ def test_host_backward_incremental_matches_oracle():
     for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
         err = np.abs(got.float().numpy() - ref) / (2e-2 + 2e-2 * np.abs(ref))
         assert float(err.max()) <= 1.0
+
+
+WA = [
+    # (B, Hq, Hkv, N, d, window, anchor period, P, kv heads per group)
+    (1, 8, 4, 1024, 128, 300, 256, 4, 0),
+    (2, 4, 2, 768, 64, 100, 512, 3, 1),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,W,A,P,kvg", WA)
+def test_host_window_anchor_is_bit_identical_to_device(B, Hq, Hkv, N, d, W, A, P, kvg):
+    R = ra()
+    w = W_(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, W=W, A=A, P=P)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    do, dl = R.ring_attn_fwd_window_anchor(q, k, v, window=W, anchor_period=A, P=P, chunk=w.chunk, scale=w.scale)
+    hq, hk, hv = (_host(x) for x in (q, k, v))
+    ho, hl = R.ring_attn_fwd_window_anchor_host(hq, hk, hv, window=W, anchor_period=A, P=P, chunk=w.chunk,
+                                                scale=w.scale, kv_heads_per_group=kvg)
+    assert R.ring_attn_sync_status() == 0
+    assert torch.equal(ho.view(torch.int16), do.cpu().view(torch.int16))
+    assert torch.equal(hl, dl.cpu())
+
+
+def W_(B, Hq, Hkv, N, d, W, A, P):
+    return workloads.small(B=B, Hq=Hq, Hkv=Hkv, N_q=N, d=d, causal=False, P=P, seed=1000 + N + W, window=W,
+                           anchor_period=A)
