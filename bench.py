@@ -53,20 +53,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel, from ncu captures (profiles/), keyed by workload, with the hash of
 # the kernel sources they were taken on.  A stale hash reports null.
 NCU_TRAFFIC = {
-    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.830061 GB read + 0.253966 GB written.
-    "llama7b_prefill_N32768": {"bytes": 1.08402688e9, "src": "bec148d66a3c98b0"},
-    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073925 GB read + 0.004619 GB written.
-    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.07854464e9, "src": "ffc6d1b8e6968136"},
+    # profiles/fwd_sm100_llama7b_prefill_N32768.md: 0.829952 GB read + 0.254706 GB written.
+    "llama7b_prefill_N32768": {"bytes": 1.084657920e9, "src": "d8709868bf1b4f82"},
+    # profiles/decode_sm100_Nq1_Nkv65536.md: 1.073960 GB read + 0.005652 GB written.
+    "cache_idx_decode_Nq1_Nkv65536": {"bytes": 1.079611648e9, "src": "8331446299cfbe48"},
     # The full-length decodes scale the quarter-length captures by their 4x KV
     # length (traffic is K/V streaming, proportional to N_kv).
-    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.07854464e9, "src": "ffc6d1b8e6968136"},
-    # profiles/decode_f8_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537022 GB read + 0.003748 GB written.
-    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.540770304e9, "src": "ffc6d1b8e6968136"},
-    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.540770304e9, "src": "ffc6d1b8e6968136"},
+    "cache_idx_decode_Nq1_Nkv262144": {"bytes": 4 * 1.079611648e9, "src": "8331446299cfbe48"},
+    # profiles/decode_f8_sm100_Nq1_Nkv65536.md (FP8 cache): 0.537050 GB read + 0.003901 GB written.
+    "cache_idx_decode_fp8kv_Nq1_Nkv65536": {"bytes": 0.540951296e9, "src": "8331446299cfbe48"},
+    "cache_idx_decode_fp8kv_Nq1_Nkv262144": {"bytes": 4 * 0.540951296e9, "src": "8331446299cfbe48"},
     # profiles/bwd_sm100_llama7b_prefill_N32768.md: one backward step, one capture
-    # per kernel (prep, dK/dV, dQ): 0.541 + 0.011, 1.084 + 0.508, 1.084 + 0.255 GB
+    # per kernel (prep, dK/dV, dQ): 0.541 + 0.010, 1.087 + 0.509, 1.086 + 0.255 GB
     # read + written.
-    "llama7b_prefill_N32768 bwd": {"bytes": 3.48383488e9, "src": "34dfa46d381e0880"},
+    "llama7b_prefill_N32768 bwd": {"bytes": 3.487720704e9, "src": "fc202d6b900047b1"},
 }
 
 
